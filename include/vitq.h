@@ -1,0 +1,211 @@
+/*
+ * vitq — FP8 ViT vision-tower forward pass for NVIDIA B200 (sm_100a).
+ *
+ * C ABI of libvitq.so.  Every computation runs in CUDA kernels of this library
+ * on the caller's stream; there is no host fallback.
+ *
+ * Conventions for every entry point
+ * ---------------------------------
+ *  - Pointers are DEVICE pointers unless a parameter says "host".  The caller
+ *    owns all memory; the library never allocates, frees or synchronises the
+ *    host (except vitq_get_device_error, which reads a device word).
+ *  - bf16 tensors are passed as `const void*` / `void*` holding IEEE bfloat16
+ *    values; FP8 codes are OCP E4M3 ("E4M3FN") bytes; scales are fp32.
+ *  - Matrices are row-major.  Activation FP8 codes are [M, K] (K contiguous);
+ *    activation scales are kb-major: s[kb * lds + m] for K block kb = k / 128
+ *    (one scale per row per 128 columns, the last block may be shorter).
+ *    Weight codes are [N, K]; weight scales are [ceil(N/128), ceil(K/128)].
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).
+ *  - Arguments are validated on the host before anything is launched; on an
+ *    error nothing is launched and a vitq_status below is returned.
+ *  - Pointers passed to the GEMM / attention paths must be 16-byte aligned.
+ *
+ * Sources (web pages; the section named is where each step is described):
+ *  [FRT] "Qwen3-VL-8B on RTX 5090 (NVFP4 language stack + FP8 ViT)"
+ *  [VE]  "spark_model/layers/vision_encoder.rs" (struct definitions)
+ *  [TRT] "qwen3_omni: record why FP8 is not shipped" (FP8 scale amax / 448)
+ */
+#ifndef VITQ_H_
+#define VITQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  VITQ_OK = 0,
+  VITQ_ERR_INVALID_ARG = 1,   /* null pointer, negative count, bad flag */
+  VITQ_ERR_SHAPE = 2,         /* unsupported dimension (K % 16, odd grid for the merger, ...) */
+  VITQ_ERR_ALIGN = 3,         /* pointer not 16-byte aligned */
+  VITQ_ERR_ARCH = 4,          /* current device is not sm_100 */
+  VITQ_ERR_CUDA = 5,          /* a CUDA call or kernel launch failed */
+  VITQ_ERR_WORKSPACE = 6,     /* workspace smaller than the *_workspace_bytes figure */
+  VITQ_ERR_DEVICE_TIMEOUT = 7 /* a kernel's bounded pipeline wait expired (see vitq_get_device_error) */
+} vitq_status;
+
+/* Model dimensions (Qwen3-VL vision tower: [FRT] section 3, [VE] VisionEncoder). */
+#define VITQ_HIDDEN 1152
+#define VITQ_HEADS 16
+#define VITQ_HEAD_DIM 72
+#define VITQ_MLP 4304
+#define VITQ_QKV 3456
+#define VITQ_MERGE_IN 4608
+#define VITQ_OUT_HIDDEN 2048
+#define VITQ_BLOCKS 27
+#define VITQ_MAX_IMAGES 64
+
+/* Weights of one ViT block ([VE] ViTBlock): LayerNorm gamma/beta and biases are
+ * bf16; each linear is FP8 codes [out, in] plus fp32 128x128 block scales. */
+typedef struct {
+  const void* norm1_w; const void* norm1_b;                   /* [1152] */
+  const uint8_t* qkv_q; const float* qkv_s; const void* qkv_b;  /* [3456,1152], [27,9], [3456] */
+  const uint8_t* proj_q; const float* proj_s; const void* proj_b; /* [1152,1152], [9,9], [1152] */
+  const void* norm2_w; const void* norm2_b;                   /* [1152] */
+  const uint8_t* fc1_q; const float* fc1_s; const void* fc1_b;  /* [4304,1152], [34,9], [4304] */
+  const uint8_t* fc2_q; const float* fc2_s; const void* fc2_b;  /* [1152,4304], [9,34], [1152] */
+} vitq_block_weights;
+
+/* Weights of one 2x2 patch merger ([VE] MergerLayer). */
+typedef struct {
+  const void* norm_w; const void* norm_b;                     /* [4608] */
+  const uint8_t* fc1_q; const float* fc1_s; const void* fc1_b;  /* [4608,4608], [36,36], [4608] */
+  const uint8_t* fc2_q; const float* fc2_s; const void* fc2_b;  /* [2048,4608], [16,36], [2048] */
+} vitq_merger_weights;
+
+/* Whole tower ([VE] VisionEncoder): 27 blocks and 4 mergers (after blocks 8, 16, 24, 27). */
+typedef struct {
+  vitq_block_weights blocks[VITQ_BLOCKS];
+  vitq_merger_weights mergers[4];
+} vitq_tower_weights;
+
+/* ---------------------------------------------------------------- stages */
+
+/* 1x128 FP8 activation quantisation ([FRT] s3 "per-token / per-128-K-block FP8
+ * activation quant"; scale convention [TRT]).  x: bf16 [M, ldx] (first K
+ * columns used).  For each row m and K block kb: s = amax / 448 (fp32 IEEE
+ * division), q = E4M3_RNE_satfinite(x / s); a zero scale gives zero codes.
+ * Outputs q [M, K] and s[kb * lds + m].  K % 16 == 0, lds >= M. */
+int vit_quant_act(const void* x, int M, int K, int ldx, uint8_t* q, float* s, int lds, void* stream);
+
+/* 128x128-block FP8 weight quantisation (same convention, one scale per block).
+ * w: bf16 [N, K] -> q [N, K], s [ceil(N/128), ceil(K/128)].  Set-up step. */
+int vit_quant_weight(const void* w, int N, int K, uint8_t* q, float* s, void* stream);
+
+/* LayerNorm (biased variance, eps) with the bf16 result quantised as in
+ * vit_quant_act ([FRT] s3 layer_norm_to_fp8_block128: the bf16 normalised
+ * activation never goes to HBM).  Statistics and the affine step in fp64,
+ * one rounding to bf16.  x: bf16 [M, ldx]; gamma/beta bf16 [K]; K <= 4608. */
+int vit_ln_quant(const void* x, int M, int K, int ldx, const void* gamma, const void* beta, float eps,
+                 uint8_t* q, float* s, int lds, void* stream);
+
+/* GELU(tanh) of a bf16 activation, rounded to bf16, quantised as in
+ * vit_quant_act ([FRT] s3 gelu_tanh_to_fp8_block128).  f: bf16 [M, ldf]. */
+int vit_gelu_quant(const void* f, int M, int K, int ldf, uint8_t* q, float* s, int lds, void* stream);
+
+/* FP8 W8A8 block-scaled GEMM with fused bias and residual ([FRT] s1 "FP8
+ * block-128 ViT GEMMs", "bias adds fused"; [VE] vision_gemm_bias):
+ *   C[m,n] = bf16( sum_kb sA[kb*ldsA+m] * sW[(n/128)*ceil(K/128)+kb] * sum_{k in kb} A[m,k] W[n,k]
+ *                  + bias[n] + residual[m,n] )
+ * A: E4M3 [M, K]; W: E4M3 [N, K]; bias bf16 [N] or NULL; residual bf16 [M, N]
+ * or NULL (may equal C); C bf16 [M, N].  K % 16 == 0, N % 8 == 0, ldsA >= M.
+ * The K tail (K % 128) is zero-filled in shared memory, so K needs no padding. */
+int fp8_block_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W, const float* sW,
+                   const void* bias, const void* residual, void* C, int M, int N, int K, void* stream);
+
+/* 2D rotary table ([FRT] s3 "2D rotate_half RoPE"; [VE] rope_inv_freq, head_dim/4
+ * entries).  pos_hw: int32 [n][2] (row, col) per token.  Output cos_sin fp32
+ * [n][72]: cos of the 36 angles then their sines; angle j = row * f_j for
+ * j < 18 and col * f_(j-18) otherwise, f_i = theta^(-2i/36).  fp64 inside. */
+int vit_rope_table(const int32_t* pos_hw, int n_tokens, float theta, float* cos_sin, void* stream);
+
+/* Flag for vit_rope2d / vit_attention_varlen: the v part of qkv is (made) fp16.
+ * v comes out of a bf16 GEMM, so bf16 -> fp16 is exact (|v| < 65504), and the
+ * attention then runs its P.V product with fp16 P (11 significant bits instead
+ * of 8) at the same tensor-core rate. */
+#define VITQ_V_FP16 1
+
+/* Apply the rotary in place to the q and k parts of qkv bf16 [n, 3, 16, 72]:
+ * pairs (j, j+36): x'_j = x_j cos - x_(j+36) sin, x'_(j+36) = x_(j+36) cos + x_j sin,
+ * fp32 arithmetic, one rounding to bf16.  flags = VITQ_V_FP16 also converts the
+ * v part to fp16 in place; flags = 0 leaves it untouched. */
+int vit_rope2d(void* qkv, int n_tokens, const float* cos_sin, int flags, void* stream);
+
+/* Patch positions of packed images ([FRT] s5: one attention window per image).
+ * grid_hw: HOST int32 [n_images][2] (h, w).  Writes pos_hw int32 [n][2] and
+ * cu_seqlens int32 [n_images + 1].  Token order: 2x2-block order for even
+ * grids (the merger's 4 neighbours are consecutive rows), row-major otherwise. */
+int vit_positions(const int32_t* grid_hw, int n_images, int32_t* pos_hw, int32_t* cu_seqlens,
+                  void* stream);
+
+/* Block-diagonal non-causal attention ([FRT] s1/s3 "FA2 (full, bidirectional)",
+ * s5 cu_seqlens).  qkv: bf16 [n_tokens, 3, 16, 72] (rotary already applied);
+ * cu_seqlens int32 [n_seqs + 1] with cu[0] = 0, cu[n_seqs] = n_tokens;
+ * max_seqlen >= every segment length.  out: bf16 [n_tokens, 1152], head h in
+ * columns h*72 .. h*72+71.  qkv must be 16-byte aligned.  flags: 0 = v is bf16
+ * and P is rounded to bf16 for P.V (flash-attention bf16 numerics);
+ * VITQ_V_FP16 = v is fp16 (see vit_rope2d) and P is rounded to fp16. */
+int vit_attention_varlen(const void* qkv, int n_tokens, const int32_t* cu_seqlens, int n_seqs,
+                         int max_seqlen, float softmax_scale, int flags, void* out, void* stream);
+
+/* ---------------------------------------------------------------- layers */
+
+/* One ViT block in place on x bf16 [n_tokens, 1152] ([FRT] s3 per-block chain):
+ * LN1+quant -> QKV GEMM+bias -> RoPE -> attention -> quant -> proj GEMM+bias+x
+ * -> LN2+quant -> fc1 GEMM+bias -> GELU+quant -> fc2 GEMM+bias+residual.
+ * cos_sin from vit_rope_table; ws >= vitq_block_workspace_bytes(n_tokens). */
+int vit_block_forward(const vitq_block_weights* w, void* x, int n_tokens, const int32_t* cu_seqlens,
+                      int n_seqs, int max_seqlen, const float* cos_sin, void* ws, size_t ws_bytes,
+                      void* stream);
+size_t vitq_block_workspace_bytes(int n_tokens);
+
+/* 2x2 spatial merger ([FRT] s3 "2x2 patch merger"; [VE] MergerLayer): rows
+ * 4i..4i+3 of x bf16 [n_tokens, 1152] form one 4608 row; LayerNorm(4608)+quant
+ * -> fc1 4608->4608 + bias -> GELU+quant -> fc2 4608->2048 + bias.
+ * out: bf16 [n_tokens/4, 2048].  n_tokens % 4 == 0. */
+int vit_merger_forward(const vitq_merger_weights* w, const void* x, int n_tokens, void* out, void* ws,
+                       size_t ws_bytes, void* stream);
+size_t vitq_merger_workspace_bytes(int n_tokens);
+
+/* The 27-block tower over packed images with DeepStack taps ([FRT] s3 "DeepStack
+ * taps at layers 8 / 16 / 24", [VE] deepstack_indexes [8,16,24] + final merger).
+ * x: bf16 [n, 1152] patch embeddings, overwritten with the block-27 output.
+ * grid_hw: HOST int32 [n_images][2], every h and w even.  taps[t]: bf16
+ * [n/4, 2048] outputs of merger t (after blocks 8, 16, 24, 27).
+ * ws >= vitq_tower_workspace_bytes(n, n_images). */
+int vit_tower_forward(const vitq_tower_weights* w, void* x, const int32_t* grid_hw, int n_images,
+                      void* const* taps, void* ws, size_t ws_bytes, void* stream);
+size_t vitq_tower_workspace_bytes(int n_tokens_max, int n_images_max);
+
+/* ---------------------------------------------------------------- status */
+
+/* Reads and clears the device error word after synchronising `stream`:
+ * 0 = none, VITQ_ERR_DEVICE_TIMEOUT = a bounded pipeline wait expired. */
+int vitq_get_device_error(void* stream);
+const char* vitq_status_string(int status);
+/* Number of kernel launches issued by this library since load (diagnostic). */
+unsigned long long vitq_launch_count(void);
+
+/* Launch timing.  Between vitq_profile_start and vitq_profile_stop every kernel
+ * launch of this library is bracketed by a CUDA event pair on its stream (not
+ * for use during stream capture).  vitq_profile_stop waits for the events and
+ * returns the number of records; vitq_profile_get returns record i: the kernel
+ * name (static string), its device time in ms, and its algorithmic FLOPs and
+ * HBM bytes (0 where the host does not know them). */
+void vitq_profile_start(void);
+int vitq_profile_stop(void);
+int vitq_profile_get(int i, const char** name, float* ms, double* flops, double* bytes);
+
+/* Runs a one-CTA kernel whose pipeline wait can never complete, with a limit of
+ * limit_us microseconds (1..1e6): the wait gives up, sets the device error word
+ * and the kernel returns, so vitq_get_device_error then reports
+ * VITQ_ERR_DEVICE_TIMEOUT.  Checks the timeout path; hangs nothing. */
+int vitq_selftest_wait_timeout(int limit_us, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VITQ_H_ */

@@ -1,0 +1,521 @@
+// Memory-bound kernels of the ViT block: FP8 block-128 activation quantisation
+// (standalone, fused after LayerNorm, fused after GELU), 128x128 weight
+// quantisation, the 2D rotary table and its in-place application, and the
+// per-patch (row, col) positions of packed images.
+//
+// Quantisation convention ("Qwen3-VL-8B on RTX 5090", section 3, fused
+// per-token / per-128-K-block FP8 activation quant; scale = amax / 448 as in
+// "qwen3_omni: record why FP8 is not shipped", recipe): for each row and each
+// group of 128 columns, s = amax / 448 (IEEE fp32 division) and
+// code = E4M3_RNE_satfinite(y / s) (IEEE fp32 division).  A zero scale gives
+// zero codes.  Scales are stored kb-major: s[kb * lds + row].
+#include "internal.h"
+#include "ptx.cuh"
+
+#include <cuda_fp16.h>
+
+namespace vitq {
+
+namespace {
+
+constexpr float kE4M3Max = 448.0f;
+
+// The quotient y / s that decides an E4M3 code.  The code depends only on which
+// side of an E4M3 rounding midpoint fl(y / s) lies; y * fl(1 / s) is within a
+// few ulps of fl(y / s), so the exact IEEE division is taken only when that
+// product lies within 16 ulps of a midpoint (mantissa tail 0x80000) or below
+// the normal E4M3 range.  The result therefore always encodes like fl(y / s).
+__device__ __forceinline__ float e4m3_quotient(float y, float s, float r) {
+  float q = y * r;
+  const uint32_t b = __float_as_uint(q) & 0x7FFFFFFFu;
+  const int mid = (int)(b & 0xFFFFFu) - 0x80000;
+  if (b < 0x3C800000u || (mid <= 16 && mid >= -16)) q = __fdiv_rn(y, s);
+  return q;
+}
+
+// Quantise 8 consecutive values of one 128-column group given the group scale.
+__device__ __forceinline__ uint2 quant8(const float (&v)[8], float s) {
+  uint32_t c[4] = {0u, 0u, 0u, 0u};
+  if (s > 0.f) {
+    const float r = __frcp_rn(s);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      c[i] = cvt_e4m3x2(e4m3_quotient(v[2 * i], s, r), e4m3_quotient(v[2 * i + 1], s, r));
+  }
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+
+// Max over the 16 lanes of a half warp.
+__device__ __forceinline__ float half_warp_max(float v) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+__device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float (&v)[8]) {
+  unpack8(*reinterpret_cast<const uint4*>(p), v);
+}
+
+// Exact value of a bf16 bit pattern as fp64, by moving its fields (zero and
+// bf16 subnormals, below 1.2e-38, give 0).
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t h) {
+  const uint32_t e = (h >> 7) & 0xFFu;
+  uint64_t bits = (uint64_t)(h & 0x8000u) << 48;
+  if (e) bits |= ((uint64_t)(e + 896u) << 52) | ((uint64_t)(h & 0x7Fu) << 45);
+  return __longlong_as_double((long long)bits);
+}
+
+// Distance from y to the nearest bf16 rounding midpoint, and its bf16 rounding.
+// Returns false when y is too small for the fp32 test (|y| < 2^-100).
+__device__ __forceinline__ bool bf16_round_margin(float y, float* yr, float* dist) {
+  const uint32_t ey = __float_as_uint(y) & 0x7F800000u;
+  *yr = __bfloat162float(__float2bfloat16_rn(y));
+  if (ey < (27u << 23)) return false;
+  const float half = __uint_as_float(ey - (8u << 23));  // half a bf16 ulp in y's binade
+  *dist = half - fabsf(y - *yr);
+  return true;
+}
+
+// Lane layout shared by the row kernels: a warp covers 256 columns per step;
+// lanes 0-15 hold group 2*step, lanes 16-31 group 2*step+1, 8 columns each.
+__device__ __forceinline__ int lane_col(int step, int lane) { return step * 256 + lane * 8; }
+
+// Group amax over the half warp, scale, codes and scale store for one step.
+__device__ __forceinline__ void quant_store(const float (&v)[8], bool ok, int lane, int row, int col, int K,
+                                            uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+  a = half_warp_max(a);
+  const float sc = __fdiv_rn(a, kE4M3Max);
+  if (ok) {
+    *reinterpret_cast<uint2*>(q + (size_t)row * K + col) = quant8(v, sc);
+    if ((lane & 15) == 0) s[(size_t)(col >> 7) * lds + row] = sc;
+  }
+}
+
+// ------------------------------------------------------------ activation quant
+// One warp per row; every load of the row is issued before any use.
+
+template <int ITERS>
+__global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ x, int M, int K, int ldx,
+                                 uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  uint4 raw[ITERS];
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int col = lane_col(it, lane);
+    raw[it] = col < K ? *reinterpret_cast<const uint4*>(x + (size_t)row * ldx + col) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int col = lane_col(it, lane);
+    float v[8];
+    unpack8(raw[it], v);
+    quant_store(v, col < K, lane, row, col, K, q, s, lds);
+  }
+}
+
+// --------------------------------------------------------- LayerNorm + quant
+// One warp per row held in registers.  The statistics are exact fp64 sums of
+// the bf16 inputs (sum and sum of squares); the normalised value is evaluated
+// in fp32 and, when it lies within its error bound of a bf16 rounding
+// midpoint, recomputed in fp64, so the bf16 result is the rounding of the fp64
+// value (x - mean) * rstd * gamma + beta.
+
+template <int ITERS>
+__global__ void ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
+                                const __nv_bfloat16* __restrict__ gamma,
+                                const __nv_bfloat16* __restrict__ beta, int M, int K, double eps,
+                                uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;
+  uint4 raw[ITERS];
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int col = lane_col(it, lane);
+    raw[it] = col < K ? *reinterpret_cast<const uint4*>(x + (size_t)row * ldx + col) : make_uint4(0, 0, 0, 0);
+  }
+  double s1 = 0.0, s2 = 0.0;
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const uint32_t w[4] = {raw[it].x, raw[it].y, raw[it].z, raw[it].w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const double a = bf16_bits_to_f64(w[i] & 0xFFFFu), b = bf16_bits_to_f64(w[i] >> 16);
+      s1 += a + b;
+      s2 = fma(a, a, fma(b, b, s2));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+  }
+  const double mean = s1 / (double)K;
+  const double var = fmax(s2 / (double)K - mean * mean, 0.0);
+  const double rstd = 1.0 / sqrt(var + eps);
+  const float mh = (float)mean, ml = (float)(mean - (double)mh), r32 = (float)rstd;
+#pragma unroll
+  for (int it = 0; it < ITERS; ++it) {
+    const int col = lane_col(it, lane);
+    const bool ok = col < K;
+    float v[8];
+    unpack8(raw[it], v);
+    if (ok) {
+      float g[8], b[8];
+      load8_bf16(gamma + col, g);
+      load8_bf16(beta + col, b);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float t = ((v[i] - mh) - ml) * r32;
+        const float y = fmaf(t, g[i], b[i]);
+        float yr, dist;
+        const float err = (fabsf(t * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;  // 2^-20
+        if (!bf16_round_margin(y, &yr, &dist) || dist <= err) {
+          const double yd = ((double)v[i] - mean) * rstd * (double)g[i] + (double)b[i];
+          yr = __bfloat162float(__double2bfloat16(yd));
+        }
+        v[i] = yr;
+      }
+    }
+    quant_store(v, ok, lane, row, col, K, q, s, lds);
+  }
+}
+
+// ------------------------------------------------------------- GELU + quant
+// GELU(tanh) = 0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)), u = sqrt(2/pi)(x + 0.044715 x^3).
+// The fp32 sigmoid form (hardware exp2 and reciprocal) has no cancellation and a
+// relative error below 2^-16 for x >= -9; when its result lies within that bound
+// of a bf16 rounding midpoint, or x < -9, the value is recomputed in fp64 in the
+// tanh form, so the bf16 result is the rounding of the fp64 GELU.
+
+__device__ __forceinline__ float gelu_tanh_bf16(float x) {
+  const float u = x * fmaf(0.035677408136300125f, x * x, 0.7978845608028654f);
+  float e, rc;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-2.8853900817779268f * u));   // exp(-2u)
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.0f + e));
+  const float g = x * rc;
+  float gr, dist;
+  if (x < -9.0f || !bf16_round_margin(g, &gr, &dist) || dist <= fabsf(g) * 1.52587890625e-05f) {  // 2^-16
+    const double xd = (double)x;
+    const double ud = 0.79788456080286535588 * (xd + 0.044715 * xd * xd * xd);
+    gr = __bfloat162float(__double2bfloat16(0.5 * xd * (1.0 + tanh(ud))));
+  }
+  return gr;
+}
+
+__global__ void gelu_quant_kernel(const __nv_bfloat16* __restrict__ f, int M, int K, int ldf,
+                                  uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+  const int steps = (K + 255) / 256;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= M * steps) return;
+  const int row = warp / steps;
+  const int st = warp - row * steps;
+  const int col = lane_col(st, lane);
+  const bool ok = col < K;
+  float v[8];
+  if (ok) {
+    load8_bf16(f + (size_t)row * ldf + col, v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = gelu_tanh_bf16(v[i]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+  }
+  quant_store(v, ok, lane, row, col, K, q, s, lds);
+}
+
+// ------------------------------------------------------------ weight quant
+// One CTA (256 threads) per 128x128 block of W [N, K].
+
+__global__ void quant_weight_kernel(const __nv_bfloat16* __restrict__ w, int N, int K,
+                                    uint8_t* __restrict__ q, float* __restrict__ s) {
+  const int nb = blockIdx.y, kb = blockIdx.x;
+  const int nkb = gridDim.x;
+  const int t = threadIdx.x;
+  // 128 rows x 16 chunks of 8 columns = 2048 chunks, 8 per thread.
+  float a = 0.f;
+  for (int c = t; c < 2048; c += 256) {
+    const int r = nb * 128 + (c >> 4);
+    const int col = kb * 128 + (c & 15) * 8;
+    if (r < N && col < K) {
+      float v[8];
+      load8_bf16(w + (size_t)r * K + col, v);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
+    }
+  }
+  __shared__ float red[8];
+  a = warp_max(a);
+  if ((t & 31) == 0) red[t >> 5] = a;
+  __syncthreads();
+  if (t < 32) {
+    float b = t < 8 ? red[t] : 0.f;
+    b = warp_max(b);
+    if (t == 0) red[0] = b;
+  }
+  __syncthreads();
+  const float sc = __fdiv_rn(red[0], kE4M3Max);
+  if (t == 0) s[nb * nkb + kb] = sc;
+  for (int c = t; c < 2048; c += 256) {
+    const int r = nb * 128 + (c >> 4);
+    const int col = kb * 128 + (c & 15) * 8;
+    if (r < N && col < K) {
+      float v[8];
+      load8_bf16(w + (size_t)r * K + col, v);
+      *reinterpret_cast<uint2*>(q + (size_t)r * K + col) = quant8(v, sc);
+    }
+  }
+}
+
+// --------------------------------------------------------------- 2D rotary
+// Table layout: cos_sin[t * 72 + j] = cos(angle_j), cos_sin[t * 72 + 36 + j] = sin(angle_j),
+// angle_j = row * f_j (j < 18), col * f_(j-18) (18 <= j < 36), f_i = theta^(-2i/36).
+
+__global__ void rope_table_kernel(const int32_t* __restrict__ pos, int n, double theta,
+                                  float* __restrict__ cs) {
+  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= n * 36) return;
+  const int t = idx / 36, j = idx - t * 36;
+  const int i = j < 18 ? j : j - 18;
+  const double f = pow(theta, -2.0 * (double)i / 36.0);
+  const double p = (double)pos[2 * t + (j < 18 ? 0 : 1)];
+  double sn, cn;
+  sincos(p * f, &sn, &cn);
+  cs[(size_t)t * 72 + j] = (float)cn;
+  cs[(size_t)t * 72 + 36 + j] = (float)sn;
+}
+
+// One CTA per token, one thread per 8-element chunk.  Chunks 0..287 are the
+// token's q and k heads (9 per head): x'_j = x_j c_j - x_(j+36) s_j,
+// x'_(j+36) = x_(j+36) c_j + x_j s_j; the partner elements of chunk cc live in
+// two neighbouring chunks A (elements 4..7) and B (elements 0..3).  Chunks
+// 288..431 are the v heads, converted to fp16 in place when v_to_f16 (bf16 ->
+// fp16 is exact for |v| < 65504).  All reads happen before the barrier and all
+// writes after it, so the in-place update never reads a rotated value.
+__global__ void __launch_bounds__(432) rope_apply_kernel(__nv_bfloat16* __restrict__ qkv,
+                                                         const float* __restrict__ cs, int v_to_f16) {
+  const int t = blockIdx.x;
+  const int c = threadIdx.x;
+  __nv_bfloat16* base = qkv + (size_t)t * 3456;
+  uint4 out = make_uint4(0, 0, 0, 0);
+  __nv_bfloat16* dst = nullptr;
+  if (c < 288) {
+    const int slot = c / 9, cc = c - slot * 9;
+    const __nv_bfloat16* head = base + slot * 72;
+    int ca, cb, k0, k1;   // partner chunks, cos/sin offsets of elements 0..3 and 4..7
+    if (cc < 4) {
+      ca = cc + 4; cb = cc + 5; k0 = 8 * cc; k1 = 8 * cc + 4;
+    } else if (cc == 4) {
+      ca = 8; cb = 0; k0 = 32; k1 = 0;
+    } else {
+      ca = cc - 5; cb = cc - 4; k0 = 8 * cc - 36; k1 = 8 * cc - 32;
+    }
+    float x[8], pa[8], pb[8];
+    load8_bf16(head + cc * 8, x);
+    load8_bf16(head + ca * 8, pa);
+    load8_bf16(head + cb * 8, pb);
+    const float* tc = cs + (size_t)t * 72;
+    const float4 c0 = __ldg(reinterpret_cast<const float4*>(tc + k0));
+    const float4 c1 = __ldg(reinterpret_cast<const float4*>(tc + k1));
+    const float4 s0 = __ldg(reinterpret_cast<const float4*>(tc + 36 + k0));
+    const float4 s1 = __ldg(reinterpret_cast<const float4*>(tc + 36 + k1));
+    const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+    const float pv[8] = {pa[4], pa[5], pa[6], pa[7], pb[0], pb[1], pb[2], pb[3]};
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool first_half = cc < 4 || (cc == 4 && i < 4);   // element j < 36
+      o[i] = first_half ? fmaf(x[i], cv[i], -pv[i] * sv[i]) : fmaf(x[i], cv[i], pv[i] * sv[i]);
+    }
+    out.x = pack_bf16x2(o[0], o[1]);
+    out.y = pack_bf16x2(o[2], o[3]);
+    out.z = pack_bf16x2(o[4], o[5]);
+    out.w = pack_bf16x2(o[6], o[7]);
+    dst = base + slot * 72 + cc * 8;
+  } else if (v_to_f16) {
+    dst = base + 2304 + (c - 288) * 8;
+    float v[8];
+    load8_bf16(dst, v);
+    __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
+    __half2 h2 = __floats2half2_rn(v[4], v[5]), h3 = __floats2half2_rn(v[6], v[7]);
+    out.x = *reinterpret_cast<uint32_t*>(&h0);
+    out.y = *reinterpret_cast<uint32_t*>(&h1);
+    out.z = *reinterpret_cast<uint32_t*>(&h2);
+    out.w = *reinterpret_cast<uint32_t*>(&h3);
+  }
+  __syncthreads();
+  if (dst) *reinterpret_cast<uint4*>(dst) = out;
+}
+
+// --------------------------------------------------------------- positions
+// Token order inside an h x w image: 2x2-block order for even grids (block
+// (br, bc) row-major, inside it (0,0) (0,1) (1,0) (1,1)), row-major otherwise.
+
+__global__ void positions_kernel(GridList grids, int n_total, int32_t* __restrict__ pos,
+                                 int32_t* __restrict__ cu) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t == 0) {
+    int acc = 0;
+    cu[0] = 0;
+    for (int i = 0; i < grids.n; ++i) {
+      acc += grids.hw[2 * i] * grids.hw[2 * i + 1];
+      cu[i + 1] = acc;
+    }
+  }
+  if (t >= n_total) return;
+  int start = 0, img = 0;
+  for (; img < grids.n; ++img) {
+    const int len = grids.hw[2 * img] * grids.hw[2 * img + 1];
+    if (t < start + len) break;
+    start += len;
+  }
+  const int h = grids.hw[2 * img], w = grids.hw[2 * img + 1];
+  const int p = t - start;
+  int r, c;
+  if ((h & 1) == 0 && (w & 1) == 0) {
+    const int blk = p >> 2, within = p & 3;
+    const int br = blk / (w >> 1), bc = blk - br * (w >> 1);
+    r = 2 * br + (within >> 1);
+    c = 2 * bc + (within & 1);
+  } else {
+    r = p / w;
+    c = p - r * w;
+  }
+  pos[2 * t] = r;
+  pos[2 * t + 1] = c;
+}
+
+// --------------------------------------------------------------- self-test
+// Waits on an mbarrier that nothing ever arrives on, with a short limit: the
+// wait gives up, raises the device error word and the kernel returns.  Used to
+// check the timeout path without hanging anything.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait_limit(smem_u32(&bar), 0, &abort_flag, limit_ns);
+  __syncthreads();
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ launchers
+
+cudaError_t launch_selftest_wait(int limit_us, cudaStream_t st) {
+  selftest_wait_kernel<<<1, 32, 0, st>>>((unsigned long long)limit_us * 1000ull);
+  return cudaGetLastError();
+}
+
+template <int IT>
+static void qa_launch(const __nv_bfloat16* x, int M, int K, int ldx, uint8_t* q, float* s, int lds,
+                      cudaStream_t st) {
+  const int threads = 128;
+  quant_act_kernel<IT><<<(unsigned)(((long long)M * 32 + threads - 1) / threads), threads, 0, st>>>(
+      x, M, K, ldx, q, s, lds);
+}
+
+cudaError_t launch_quant_act(const __nv_bfloat16* x, int M, int K, int ldx, uint8_t* q, float* s,
+                             int lds, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  switch ((K + 255) / 256) {
+#define VITQ_QA_CASE(N) \
+  case N: qa_launch<N>(x, M, K, ldx, q, s, lds, st); break;
+    VITQ_QA_CASE(1) VITQ_QA_CASE(2) VITQ_QA_CASE(3) VITQ_QA_CASE(4) VITQ_QA_CASE(5)
+    VITQ_QA_CASE(6) VITQ_QA_CASE(7) VITQ_QA_CASE(8) VITQ_QA_CASE(9) VITQ_QA_CASE(10)
+    VITQ_QA_CASE(11) VITQ_QA_CASE(12) VITQ_QA_CASE(13) VITQ_QA_CASE(14) VITQ_QA_CASE(15)
+    VITQ_QA_CASE(16) VITQ_QA_CASE(17) VITQ_QA_CASE(18)
+#undef VITQ_QA_CASE
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+template <int IT>
+static void ln_launch(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* g,
+                      const __nv_bfloat16* b, int M, int K, double eps, uint8_t* q, float* s, int lds,
+                      cudaStream_t st) {
+  const int threads = 128;
+  ln_quant_kernel<IT><<<(unsigned)(((long long)M * 32 + threads - 1) / threads), threads, 0, st>>>(
+      x, ldx, g, b, M, K, eps, q, s, lds);
+}
+
+cudaError_t launch_ln_quant(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma,
+                            const __nv_bfloat16* beta, int M, int K, double eps, uint8_t* q,
+                            float* s, int lds, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const int it = (K + 255) / 256;
+  switch (it) {
+#define VITQ_LN_CASE(N) \
+  case N: ln_launch<N>(x, ldx, gamma, beta, M, K, eps, q, s, lds, st); break;
+    VITQ_LN_CASE(1) VITQ_LN_CASE(2) VITQ_LN_CASE(3) VITQ_LN_CASE(4) VITQ_LN_CASE(5)
+    VITQ_LN_CASE(6) VITQ_LN_CASE(7) VITQ_LN_CASE(8) VITQ_LN_CASE(9) VITQ_LN_CASE(10)
+    VITQ_LN_CASE(11) VITQ_LN_CASE(12) VITQ_LN_CASE(13) VITQ_LN_CASE(14) VITQ_LN_CASE(15)
+    VITQ_LN_CASE(16) VITQ_LN_CASE(17) VITQ_LN_CASE(18)
+#undef VITQ_LN_CASE
+    default: return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gelu_quant(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* q, float* s,
+                              int lds, cudaStream_t st) {
+  if (M == 0) return cudaSuccess;
+  const int threads = 256;
+  const long long warps = (long long)M * ((K + 255) / 256);
+  gelu_quant_kernel<<<(unsigned)((warps * 32 + threads - 1) / threads), threads, 0, st>>>(f, M, K, ldf,
+                                                                                         q, s, lds);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_weight(const __nv_bfloat16* w, int N, int K, uint8_t* q, float* s,
+                                cudaStream_t st) {
+  if (N == 0 || K == 0) return cudaSuccess;
+  dim3 grid((K + 127) / 128, (N + 127) / 128);
+  quant_weight_kernel<<<grid, 256, 0, st>>>(w, N, K, q, s);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(const int32_t* pos, int n, double theta, float* cs, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int threads = 256;
+  rope_table_kernel<<<(unsigned)(((long long)n * 36 + threads - 1) / threads), threads, 0, st>>>(
+      pos, n, theta, cs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_apply(__nv_bfloat16* qkv, int n, const float* cs, int v_to_f16, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  rope_apply_kernel<<<n, 432, 0, st>>>(qkv, cs, v_to_f16);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_positions(const GridList& g, int n_total, int32_t* pos, int32_t* cu,
+                             cudaStream_t st) {
+  const int threads = 256;
+  const int blocks = n_total > 0 ? (n_total + threads - 1) / threads : 1;
+  positions_kernel<<<blocks, threads, 0, st>>>(g, n_total, pos, cu);
+  return cudaGetLastError();
+}
+
+}  // namespace vitq

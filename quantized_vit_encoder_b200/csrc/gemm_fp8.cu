@@ -1,0 +1,302 @@
+// FP8 E4M3 W8A8 block-scaled GEMM on the sm_100a tensor cores (tcgen05 + TMEM + TMA).
+//
+//   C[m, n] = bf16( sum_kb sA[kb, m] * sW[n / 128, kb] * (A_kb[m, :] . W_kb[n, :]) + bias[n] + R[m, n] )
+//
+// "Qwen3-VL-8B on RTX 5090", sections 1 and 3: the ViT linears run as FP8
+// block-128 W8A8 GEMMs (per-token per-128-K activation scales, per-128x128
+// weight scales), with the bias adds and the residual fused into the GEMM.
+//
+// Design (B200):
+//   * persistent CTAs, one per SM, walking 128 x BN output tiles;
+//   * warp 0: TMA producer (A and W tiles of 128 K-columns into a multi-stage
+//     128B-swizzled shared-memory ring, zero fill past K / M / N);
+//   * warp 1: MMA issuer, 4 x tcgen05.mma kind::f8f6f4 (K = 32 each) per K
+//     block into one of 512/BN TMEM partial buffers;
+//   * BN/32 epilogue warps: each thread owns one output row and 128 columns,
+//     reads the K block's partial from TMEM and accumulates
+//     acc += partial * sA * sW in registers (the scales differ per K block, so
+//     the tensor core cannot accumulate across K blocks); after the last K
+//     block it adds bias and residual and stores bf16.
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace vitq {
+namespace {
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int BM = 128, BK = 128;
+  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int A_BYTES = BM * BK;
+  static constexpr int B_BYTES = BN * BK;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int NBUF = 512 / BN;
+  static constexpr int EPI_WARPS = BN / 32;
+  static constexpr int THREADS = 64 + BN;
+  static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF) * 8 + 16;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
+};
+
+struct GemmArgs {
+  const float* sA;
+  int ldsA;
+  const float* sW;
+  const __nv_bfloat16* bias;
+  const __nv_bfloat16* residual;
+  __nv_bfloat16* C;
+  int M, N, K;
+};
+
+template <int BN>
+struct GemmSmem {
+  using Cfg = GemmCfg<BN>;
+  uint8_t* base;
+  __device__ uint32_t a(int s) const { return smem_u32(base + (size_t)s * Cfg::STAGE_BYTES); }
+  __device__ uint32_t b(int s) const {
+    return smem_u32(base + (size_t)s * Cfg::STAGE_BYTES + Cfg::A_BYTES);
+  }
+  __device__ uint64_t* bars() const {
+    return reinterpret_cast<uint64_t*>(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES);
+  }
+  __device__ uint32_t full(int s) const { return smem_u32(bars() + s); }
+  __device__ uint32_t empty(int s) const { return smem_u32(bars() + Cfg::STAGES + s); }
+  __device__ uint32_t tfull(int b) const { return smem_u32(bars() + 2 * Cfg::STAGES + b); }
+  __device__ uint32_t tempty(int b) const {
+    return smem_u32(bars() + 2 * Cfg::STAGES + Cfg::NBUF + b);
+  }
+  __device__ uint32_t* tmem_holder() const {
+    return reinterpret_cast<uint32_t*>(bars() + 2 * Cfg::STAGES + 2 * Cfg::NBUF);
+  }
+  __device__ volatile int* abort_flag() const {
+    return reinterpret_cast<volatile int*>(tmem_holder() + 1);
+  }
+};
+
+template <int BN>
+__device__ void gemm_producer(const GemmSmem<BN>& sm, const CUtensorMap* tmA, const CUtensorMap* tmB,
+                              int tiles_m, int num_tiles, int nkb) {
+  using Cfg = GemmCfg<BN>;
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    const int m0 = (tile % tiles_m) * Cfg::BM;
+    const int n0 = (tile / tiles_m) * BN;
+    for (int kb = 0; kb < nkb; ++kb) {
+      if (!mbar_wait(sm.empty(stage), phase ^ 1u, sm.abort_flag())) return;
+      mbar_arrive_expect_tx(sm.full(stage), Cfg::STAGE_BYTES);
+      tma_load_2d(sm.a(stage), tmA, kb * Cfg::BK, m0, sm.full(stage));
+      tma_load_2d(sm.b(stage), tmB, kb * Cfg::BK, n0, sm.full(stage));
+      if (++stage == Cfg::STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+}
+
+template <int BN>
+__device__ void gemm_mma(const GemmSmem<BN>& sm, uint32_t tmem_base, int num_tiles, int nkb) {
+  using Cfg = GemmCfg<BN>;
+  constexpr uint32_t idesc = make_idesc(0, 0, 0, 0, 128, BN);
+  int stage = 0;
+  uint32_t phase = 0;
+  uint32_t cnt = 0;
+  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    for (int kb = 0; kb < nkb; ++kb, ++cnt) {
+      const uint32_t buf = cnt % Cfg::NBUF;
+      const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
+      if (!mbar_wait(sm.tempty(buf), aph ^ 1u, sm.abort_flag())) return;
+      tc_fence_after();
+      if (!mbar_wait(sm.full(stage), phase, sm.abort_flag())) return;
+      tc_fence_after();
+      const uint32_t a0 = sm.a(stage), b0 = sm.b(stage);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t ad = make_smem_desc(a0 + 32 * k, 16, 1024, kSwizzle128B);
+        const uint64_t bd = make_smem_desc(b0 + 32 * k, 16, 1024, kSwizzle128B);
+        mma_f8_ss(tmem_base + buf * BN, ad, bd, idesc, k > 0 ? 1u : 0u);
+      }
+      tc_commit(sm.empty(stage));
+      tc_commit(sm.tfull(buf));
+      if (++stage == Cfg::STAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+}
+
+template <int BN>
+__device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const GemmArgs& g,
+                              int tiles_m, int num_tiles, int nkb) {
+  using Cfg = GemmCfg<BN>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+  const int cg = (warp - 2) >> 2;          // which 128-column half of the tile
+  const int r_in = quad * 32 + lane;
+  uint32_t cnt = 0;
+  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    const int m0 = (tile % tiles_m) * Cfg::BM;
+    const int n0 = (tile / tiles_m) * BN;
+    const int row = m0 + r_in;
+    const int col0 = n0 + cg * 128;
+    const bool row_ok = row < g.M;
+    const bool col_ok = col0 < g.N;
+    float acc[128];
+#pragma unroll
+    for (int j = 0; j < 128; ++j) acc[j] = 0.f;
+    for (int kb = 0; kb < nkb; ++kb, ++cnt) {
+      const uint32_t buf = cnt % Cfg::NBUF;
+      const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
+      const float sa = row_ok ? __ldg(g.sA + (size_t)kb * g.ldsA + row) : 0.f;
+      const float sw = col_ok ? __ldg(g.sW + (size_t)(col0 >> 7) * nkb + kb) : 0.f;
+      const float scale = sa * sw;
+      const bool ok = mbar_wait(sm.tfull(buf), aph, sm.abort_flag());
+      if (!__all_sync(0xffffffffu, ok)) return;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + cg * 128;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint32_t r[32];
+        tmem_ld32(taddr + c * 32, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), scale, acc[c * 32 + j]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.tempty(buf));
+    }
+    if (row_ok && col_ok) {
+      __nv_bfloat16* crow = g.C + (size_t)row * g.N;
+      const __nv_bfloat16* rrow = g.residual ? g.residual + (size_t)row * g.N : nullptr;
+#pragma unroll
+      for (int c8 = 0; c8 < 16; ++c8) {
+        const int col = col0 + c8 * 8;
+        if (col < g.N) {
+          float v[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = acc[c8 * 8 + i];
+          if (g.bias) {
+            const uint4 bu = __ldg(reinterpret_cast<const uint4*>(g.bias + col));
+            const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = unpack_bf16x2(bw[i]);
+              v[2 * i] += f.x;
+              v[2 * i + 1] += f.y;
+            }
+          }
+          if (rrow) {
+            const uint4 ru = *reinterpret_cast<const uint4*>(rrow + col);
+            const uint32_t rw[4] = {ru.x, ru.y, ru.z, ru.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 f = unpack_bf16x2(rw[i]);
+              v[2 * i] += f.x;
+              v[2 * i + 1] += f.y;
+            }
+          }
+          uint4 o;
+          o.x = pack_bf16x2(v[0], v[1]);
+          o.y = pack_bf16x2(v[2], v[3]);
+          o.z = pack_bf16x2(v[4], v[5]);
+          o.w = pack_bf16x2(v[6], v[7]);
+          *reinterpret_cast<uint4*>(crow + col) = o;
+        }
+      }
+    }
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
+    fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmArgs args) {
+  using Cfg = GemmCfg<BN>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  GemmSmem<BN> sm;
+  sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nkb = (args.K + Cfg::BK - 1) / Cfg::BK;
+  const int tiles_m = (args.M + Cfg::BM - 1) / Cfg::BM;
+  const int tiles_n = (args.N + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(sm.full(s), 1);
+      mbar_init(sm.empty(s), 1);
+    }
+    for (int b = 0; b < Cfg::NBUF; ++b) {
+      mbar_init(sm.tfull(b), 1);
+      mbar_init(sm.tempty(b), Cfg::EPI_WARPS);
+    }
+    *sm.abort_flag() = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(sm.tmem_holder()), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *sm.tmem_holder();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      prefetch_tensormap(&tmA);
+      prefetch_tensormap(&tmB);
+      gemm_producer<BN>(sm, &tmA, &tmB, tiles_m, num_tiles, nkb);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) gemm_mma<BN>(sm, tmem_base, num_tiles, nkb);
+  } else {
+    gemm_epilogue<BN>(sm, tmem_base, args, tiles_m, num_tiles, nkb);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (*sm.abort_flag()) settle_pause(50000);
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 512);
+  }
+}
+
+template <int BN>
+cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
+                      cudaStream_t st) {
+  using Cfg = GemmCfg<BN>;
+  static bool attr_done = false;  // per process; the attribute is per device function
+  if (!attr_done) {
+    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)Cfg::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done = true;
+  }
+  const int tiles = ((a.M + 127) / 128) * ((a.N + BN - 1) / BN);
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  fp8_gemm_kernel<BN><<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(tmA, tmB, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fp8_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W, const float* sW,
+                            const __nv_bfloat16* bias, const __nv_bfloat16* residual, __nv_bfloat16* C,
+                            int M, int N, int K, int block_n, int num_sms, cudaStream_t st) {
+  if (M == 0 || N == 0) return cudaSuccess;
+  CUtensorMap tmA, tmB;
+  const int bn = block_n == 256 ? 256 : 128;
+  cudaError_t e = encode_tma_2d_u8(&tmA, A, K, M, 128, 128);
+  if (e != cudaSuccess) return e;
+  e = encode_tma_2d_u8(&tmB, W, K, N, 128, bn);
+  if (e != cudaSuccess) return e;
+  GemmArgs a{sA, ldsA, sW, bias, residual, C, M, N, K};
+  return bn == 256 ? launch_bn<256>(tmA, tmB, a, num_sms, st) : launch_bn<128>(tmA, tmB, a, num_sms, st);
+}
+
+}  // namespace vitq

@@ -1,0 +1,5 @@
+// Single translation unit for libvitq.so (the kernels share one device error word).
+#include "elementwise.cu"
+#include "gemm_fp8.cu"
+#include "attention.cu"
+#include "api.cu"

@@ -1,0 +1,303 @@
+"""ctypes binding of libvitq.so: the same entry points as include/vitq.h.
+
+Argument marshalling only: every step of the computation runs in the
+library's CUDA kernels.  torch supplies device memory and the current CUDA
+stream.  If the library is missing, loading raises; there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvitq.so")
+
+HIDDEN, HEADS, HEAD_DIM, MLP, QKV = 1152, 16, 72, 4304, 3456
+MERGE_IN, OUT_HIDDEN, N_BLOCKS = 4608, 2048, 27
+STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "pointer not 16-byte aligned",
+          4: "device is not sm_100", 5: "CUDA error", 6: "workspace too small",
+          7: "device pipeline wait timed out"}
+
+_vp, _i, _f, _sz = C.c_void_p, C.c_int, C.c_float, C.c_size_t
+
+
+class BlockWeights(C.Structure):
+    _fields_ = [(n, _vp) for n in (
+        "norm1_w", "norm1_b", "qkv_q", "qkv_s", "qkv_b", "proj_q", "proj_s", "proj_b",
+        "norm2_w", "norm2_b", "fc1_q", "fc1_s", "fc1_b", "fc2_q", "fc2_s", "fc2_b")]
+
+
+class MergerWeights(C.Structure):
+    _fields_ = [(n, _vp) for n in (
+        "norm_w", "norm_b", "fc1_q", "fc1_s", "fc1_b", "fc2_q", "fc2_s", "fc2_b")]
+
+
+class TowerWeights(C.Structure):
+    _fields_ = [("blocks", BlockWeights * N_BLOCKS), ("mergers", MergerWeights * 4)]
+
+
+_SIGS = {
+    "vit_quant_act": [_vp, _i, _i, _i, _vp, _vp, _i, _vp],
+    "vit_quant_weight": [_vp, _i, _i, _vp, _vp, _vp],
+    "vit_ln_quant": [_vp, _i, _i, _i, _vp, _vp, _f, _vp, _vp, _i, _vp],
+    "vit_gelu_quant": [_vp, _i, _i, _i, _vp, _vp, _i, _vp],
+    "fp8_block_gemm": [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
+    "vit_rope_table": [_vp, _i, _f, _vp, _vp],
+    "vit_rope2d": [_vp, _i, _vp, _i, _vp],
+    "vit_positions": [_vp, _i, _vp, _vp, _vp],
+    "vit_attention_varlen": [_vp, _i, _vp, _i, _i, _f, _i, _vp, _vp],
+    "vit_block_forward": [C.POINTER(BlockWeights), _vp, _i, _vp, _i, _i, _vp, _vp, _sz, _vp],
+    "vitq_block_workspace_bytes": [_i],
+    "vit_merger_forward": [C.POINTER(MergerWeights), _vp, _i, _vp, _vp, _sz, _vp],
+    "vitq_merger_workspace_bytes": [_i],
+    "vit_tower_forward": [C.POINTER(TowerWeights), _vp, _vp, _i, C.POINTER(_vp), _vp, _sz, _vp],
+    "vitq_tower_workspace_bytes": [_i, _i],
+    "vitq_get_device_error": [_vp],
+    "vitq_status_string": [_i],
+    "vitq_launch_count": [],
+    "vitq_profile_start": [],
+    "vitq_profile_stop": [],
+    "vitq_profile_get": [_i, C.POINTER(C.c_char_p), C.POINTER(C.c_float), C.POINTER(C.c_double),
+                         C.POINTER(C.c_double)],
+    "vitq_selftest_wait_timeout": [_i, _vp],
+}
+_RES = {"vitq_block_workspace_bytes": _sz, "vitq_merger_workspace_bytes": _sz,
+        "vitq_tower_workspace_bytes": _sz, "vitq_status_string": C.c_char_p,
+        "vitq_launch_count": C.c_ulonglong, "vitq_profile_start": None}
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libvitq.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(path):
+            raise RuntimeError(f"{path} is missing: build it with `python -m quantized_vit_encoder_b200.build`")
+        lib = C.CDLL(path)
+        for name, args in _SIGS.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = _RES.get(name, _i)
+        _lib = lib
+    return _lib
+
+
+class VitqError(RuntimeError):
+    pass
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        raise VitqError(f"{what}: {STATUS.get(status, status)} ({status})")
+
+
+def _p(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return C.c_void_p(s.cuda_stream)
+
+
+def launch_count() -> int:
+    return int(load().vitq_launch_count())
+
+
+def device_error(stream=None) -> int:
+    return int(load().vitq_get_device_error(_stream(stream)))
+
+
+def profile_start():
+    load().vitq_profile_start()
+
+
+def profile_stop() -> list:
+    """Per-launch records since profile_start: [(kernel name, ms, flops, bytes), ...]."""
+    lib = load()
+    n = lib.vitq_profile_stop()
+    if n < 0:
+        raise VitqError(f"vitq_profile_stop: {n}")
+    out = []
+    name, ms, fl, by = C.c_char_p(), C.c_float(), C.c_double(), C.c_double()
+    for i in range(n):
+        _check(lib.vitq_profile_get(i, C.byref(name), C.byref(ms), C.byref(fl), C.byref(by)), "vitq_profile_get")
+        out.append((name.value.decode(), float(ms.value), float(fl.value), float(by.value)))
+    return out
+
+
+def selftest_wait_timeout(limit_us: int = 20000, stream=None):
+    _check(load().vitq_selftest_wait_timeout(limit_us, _stream(stream)), "vitq_selftest_wait_timeout")
+
+
+# ---------------------------------------------------------------- stages
+
+def _scales(nkb, M, device):
+    lds = (M + 3) // 4 * 4
+    return torch.zeros((nkb, lds), dtype=torch.float32, device=device), lds
+
+
+def quant_act(x: torch.Tensor, stream=None):
+    """1x128 FP8 quantisation of bf16 x [M, K] -> (codes uint8 [M, K], scales fp32 [ceil(K/128), M_pad4])."""
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    s, lds = _scales((K + 127) // 128, M, x.device)
+    _check(load().vit_quant_act(_p(x), M, K, x.stride(0), _p(q), _p(s), lds, _stream(stream)), "vit_quant_act")
+    return q, s
+
+
+def quant_weight(w: torch.Tensor, stream=None):
+    """128x128-block FP8 quantisation of bf16 w [N, K] -> (codes [N, K], scales [ceil(N/128), ceil(K/128)])."""
+    N, K = w.shape
+    q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
+    s = torch.zeros(((N + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=w.device)
+    _check(load().vit_quant_weight(_p(w), N, K, _p(q), _p(s), _stream(stream)), "vit_quant_weight")
+    return q, s
+
+
+def ln_quant(x, gamma, beta, eps: float = 1e-6, stream=None):
+    M, K = x.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    s, lds = _scales((K + 127) // 128, M, x.device)
+    _check(load().vit_ln_quant(_p(x), M, K, x.stride(0), _p(gamma), _p(beta), eps, _p(q), _p(s), lds,
+                               _stream(stream)), "vit_ln_quant")
+    return q, s
+
+
+def gelu_quant(f, stream=None):
+    M, K = f.shape
+    q = torch.empty((M, K), dtype=torch.uint8, device=f.device)
+    s, lds = _scales((K + 127) // 128, M, f.device)
+    _check(load().vit_gelu_quant(_p(f), M, K, f.stride(0), _p(q), _p(s), lds, _stream(stream)), "vit_gelu_quant")
+    return q, s
+
+
+def fp8_block_gemm(qa, sa, qw, sw, bias=None, residual=None, out=None, stream=None):
+    """bf16 C [M, N] = block-scaled FP8 product (+ bias) (+ residual)."""
+    M, K = qa.shape
+    N = qw.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.device)
+    _check(load().fp8_block_gemm(_p(qa), _p(sa), sa.stride(0), _p(qw), _p(sw), _p(bias), _p(residual), _p(out),
+                                 M, N, K, _stream(stream)), "fp8_block_gemm")
+    return out
+
+
+def rope_table(pos_hw: torch.Tensor, theta: float = 10000.0, stream=None):
+    n = pos_hw.shape[0]
+    cs = torch.empty((n, 72), dtype=torch.float32, device=pos_hw.device)
+    _check(load().vit_rope_table(_p(pos_hw), n, theta, _p(cs), _stream(stream)), "vit_rope_table")
+    return cs
+
+
+V_FP16 = 1
+
+
+def rope2d_(qkv: torch.Tensor, cos_sin: torch.Tensor, flags: int = 0, stream=None):
+    """In-place 2D rotary on the q, k parts of qkv; flags=V_FP16 also converts v to fp16 in place."""
+    _check(load().vit_rope2d(_p(qkv), qkv.shape[0], _p(cos_sin), flags, _stream(stream)), "vit_rope2d")
+    return qkv
+
+
+def positions(grids, device="cuda", stream=None):
+    """(pos_hw int32 [n, 2], cu_seqlens int32 [n_images + 1]) for packed grids [(h, w), ...]."""
+    g = (C.c_int32 * (2 * len(grids)))(*[v for hw in grids for v in hw])
+    n = sum(h * w for h, w in grids)
+    pos = torch.empty((n, 2), dtype=torch.int32, device=device)
+    cu = torch.empty((len(grids) + 1,), dtype=torch.int32, device=device)
+    _check(load().vit_positions(C.cast(g, C.c_void_p), len(grids), _p(pos), _p(cu), _stream(stream)),
+           "vit_positions")
+    return pos, cu
+
+
+def attention_varlen(qkv, cu_seqlens, max_seqlen: int, scale: float | None = None, out=None, flags: int = 0,
+                     stream=None):
+    n = qkv.shape[0]
+    if out is None:
+        out = torch.empty((n, HIDDEN), dtype=torch.bfloat16, device=qkv.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(HEAD_DIM)
+    _check(load().vit_attention_varlen(_p(qkv), n, _p(cu_seqlens), cu_seqlens.shape[0] - 1, max_seqlen, scale,
+                                       flags, _p(out), _stream(stream)), "vit_attention_varlen")
+    return out
+
+
+# ---------------------------------------------------------------- layers
+
+class DeviceBlock:
+    """Device-resident block weights (bf16 vectors, FP8 codes, fp32 scales) and their C struct."""
+
+    def __init__(self, params: dict, device="cuda", stream=None):
+        t = {k: v.to(device) for k, v in params.items()}
+        self.t = t
+        for name in ("qkv", "proj", "fc1", "fc2"):
+            t[name + "_q"], t[name + "_s"] = quant_weight(t[name + "_w"], stream)
+        self.struct = BlockWeights(**{f: t[f].data_ptr() for f, _ in BlockWeights._fields_})
+
+
+class DeviceMerger:
+    def __init__(self, params: dict, device="cuda", stream=None):
+        t = {k: v.to(device) for k, v in params.items()}
+        self.t = t
+        for name in ("fc1", "fc2"):
+            t[name + "_q"], t[name + "_s"] = quant_weight(t[name + "_w"], stream)
+        self.struct = MergerWeights(**{f: t[f].data_ptr() for f, _ in MergerWeights._fields_})
+
+
+def block_workspace_bytes(n: int) -> int:
+    return int(load().vitq_block_workspace_bytes(n))
+
+
+def merger_workspace_bytes(n: int) -> int:
+    return int(load().vitq_merger_workspace_bytes(n))
+
+
+def tower_workspace_bytes(n: int, n_images: int) -> int:
+    return int(load().vitq_tower_workspace_bytes(n, n_images))
+
+
+def workspace(nbytes: int, device="cuda"):
+    return torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=device)
+
+
+def block_forward_(blk: DeviceBlock, x, cu_seqlens, max_seqlen, cos_sin, ws, stream=None):
+    """In-place block forward on bf16 x [n, 1152]."""
+    _check(load().vit_block_forward(C.byref(blk.struct), _p(x), x.shape[0], _p(cu_seqlens), cu_seqlens.shape[0] - 1,
+                                    max_seqlen, _p(cos_sin), _p(ws), ws.numel(), _stream(stream)),
+           "vit_block_forward")
+    return x
+
+
+def merger_forward(mg: DeviceMerger, x, ws, out=None, stream=None):
+    n = x.shape[0]
+    if out is None:
+        out = torch.empty((n // 4, OUT_HIDDEN), dtype=torch.bfloat16, device=x.device)
+    _check(load().vit_merger_forward(C.byref(mg.struct), _p(x), n, _p(out), _p(ws), ws.numel(), _stream(stream)),
+           "vit_merger_forward")
+    return out
+
+
+class DeviceTower:
+    def __init__(self, blocks, mergers):
+        self.blocks, self.mergers = blocks, mergers
+        self.struct = TowerWeights()
+        for i, b in enumerate(blocks):
+            self.struct.blocks[i] = b.struct
+        for i, m in enumerate(mergers):
+            self.struct.mergers[i] = m.struct
+
+
+def tower_forward_(tower: DeviceTower, x, grids, ws, taps=None, stream=None):
+    """In-place tower forward on bf16 x [n, 1152]; returns the four tap tensors [n/4, 2048]."""
+    n = x.shape[0]
+    if taps is None:
+        taps = [torch.empty((n // 4, OUT_HIDDEN), dtype=torch.bfloat16, device=x.device) for _ in range(4)]
+    g = (C.c_int32 * (2 * len(grids)))(*[v for hw in grids for v in hw])
+    tp = (C.c_void_p * 4)(*[t.data_ptr() for t in taps])
+    _check(load().vit_tower_forward(C.byref(tower.struct), _p(x), C.cast(g, C.c_void_p), len(grids), tp, _p(ws),
+                                    ws.numel(), _stream(stream)), "vit_tower_forward")
+    return taps

@@ -1,0 +1,256 @@
+"""GPU parity of each stage against the CPU oracle, through the C ABI.
+
+Every CUDA stage is fed the oracle's own inputs for that stage (seeded
+synthetic tensors from workloads.py).  FP8 codes and scales are compared
+bit for bit; bf16 stage outputs within rel-L2 <= 1e-2 and max-abs <= 3e-2
+(the stated per-stage tolerance).  Shapes cover several 128-tiles, ragged
+M / N / K tails, one-row and one-token cases, and the full 6256-patch sizes.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import numerics as onum
+from oracle import vit as ov
+from quantized_vit_encoder_b200 import workloads as wl
+
+pytestmark = pytest.mark.gpu
+
+REL_L2, MAX_ABS = 1e-2, 3e-2
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().float().cpu().double().numpy()
+
+
+def rel_l2(a, b):
+    a, b = np.asarray(a, np.float64), np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def assert_close(got, want, rel=REL_L2, mabs=MAX_ABS, what=""):
+    got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    assert np.all(np.isfinite(got)), what
+    r, m = rel_l2(got, want), float(np.max(np.abs(got - want))) if got.size else 0.0
+    assert r <= rel and m <= mabs, f"{what}: rel_l2={r:.3e} max_abs={m:.3e}"
+    return r, m
+
+
+def assert_codes_equal(q_gpu, s_gpu, q_ref, s_ref, what=""):
+    M = q_ref.shape[0]
+    qg = q_gpu.cpu().numpy()
+    sg = s_gpu.cpu().numpy()[:, :M]
+    bad_s = np.argwhere(sg != s_ref)
+    assert bad_s.size == 0, f"{what}: {len(bad_s)} scales differ, first {bad_s[:3].tolist()}"
+    bad_q = np.argwhere(qg != q_ref)
+    assert bad_q.size == 0, f"{what}: {len(bad_q)} codes differ, first {bad_q[:3].tolist()}"
+
+
+def bf16(shape, seed, std=1.0):
+    return wl.random_bf16(shape, seed, std)
+
+
+# ----------------------------------------------------------------- quantisation
+
+@pytest.mark.parametrize("M,K", [(1, 16), (127, 1152), (129, 4304), (300, 4608), (972, 1152), (6256, 1152)])
+def test_quant_act_bit_exact(lib, M, K):
+    from quantized_vit_encoder_b200 import vitq
+    x = bf16((M, K), 10 + M + K, 3.0)
+    q, s = vitq.quant_act(x.cuda())
+    qr, sr = ov.quant_act(f64(x))
+    assert_codes_equal(q, s, qr, sr, f"quant_act {M}x{K}")
+
+
+def test_quant_act_every_bf16_value(lib):
+    """All 65536 bf16 bit patterns (finite ones), in groups with different amax, encode bit-exactly."""
+    from quantized_vit_encoder_b200 import vitq
+    bits = np.arange(65536, dtype=np.uint32)
+    vals = onum.bf16_bits_to_f64(bits)
+    vals = vals[np.isfinite(vals)]
+    vals = vals[np.abs(vals) < 1e30]               # keep amax/448 and v/s finite in fp32
+    g = np.random.default_rng(0)
+    rows = []
+    for amax in (1.0, 448.0, 3.0e-3, 7.5e4, 1e-30):
+        v = vals[np.abs(vals) <= amax]
+        v = g.permutation(v)
+        pad = (-len(v)) % 127
+        v = np.concatenate([v, np.zeros(pad)]).reshape(-1, 127)
+        rows.append(np.concatenate([v, np.full((v.shape[0], 1), amax)], 1))
+    x = np.concatenate(rows, 0)
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    q, s = vitq.quant_act(xt.cuda())
+    qr, sr = ov.quant_act(f64(xt))
+    assert_codes_equal(q, s, qr, sr, "exhaustive")
+
+
+@pytest.mark.parametrize("N,K", [(3456, 1152), (1152, 4304), (4304, 1152), (200, 272)])
+def test_quant_weight_bit_exact(lib, N, K):
+    from quantized_vit_encoder_b200 import vitq
+    w = bf16((N, K), 20 + N, 0.02)
+    q, s = vitq.quant_weight(w.cuda())
+    qr, sr = ov.quant_weight(f64(w))
+    assert np.array_equal(s.cpu().numpy(), sr)
+    assert np.array_equal(q.cpu().numpy(), qr)
+
+
+@pytest.mark.parametrize("M,K,scale", [(1, 1152, 1.0), (129, 1152, 10.0), (972, 1152, 0.1), (301, 4608, 1.0),
+                                       (6256, 1152, 1.0)])
+def test_ln_quant_bit_exact(lib, M, K, scale):
+    from quantized_vit_encoder_b200 import vitq
+    x = bf16((M, K), 30 + M, scale)
+    g = (1 + wl.random_bf16((K,), 31, 0.02).float()).to(torch.bfloat16)
+    b = wl.random_bf16((K,), 32, 0.01)
+    q, s = vitq.ln_quant(x.cuda(), g.cuda(), b.cuda())
+    qr, sr = ov.ln_quant(f64(x), f64(g), f64(b), 1e-6)
+    assert_codes_equal(q, s, qr, sr, f"ln_quant {M}x{K}")
+
+
+@pytest.mark.parametrize("M,K", [(1, 4304), (129, 4304), (972, 4304), (100, 4608), (6256, 4304)])
+def test_gelu_quant_bit_exact(lib, M, K):
+    from quantized_vit_encoder_b200 import vitq
+    f = bf16((M, K), 40 + M, 1.5)
+    q, s = vitq.gelu_quant(f.cuda())
+    qr, sr = ov.gelu_quant(f64(f))
+    assert_codes_equal(q, s, qr, sr, f"gelu_quant {M}x{K}")
+
+
+# ----------------------------------------------------------------- GEMM
+
+GEMM_SHAPES = [
+    (1, 128, 128), (128, 128, 1152), (129, 3456, 1152), (256, 1152, 4304), (972, 4304, 1152),
+    (300, 2048, 4608), (77, 136, 272), (6256, 1152, 1152),
+]
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_fp8_gemm_matches_oracle(lib, monkeypatch, bn, M, N, K):
+    from quantized_vit_encoder_b200 import vitq
+    monkeypatch.setenv("VITQ_GEMM_BN", str(bn))
+    a = bf16((M, K), 50 + M, 1.0)
+    w = bf16((N, K), 51 + N, 0.02)
+    bias = bf16((N,), 52, 0.01)
+    res = bf16((M, N), 53, 1.0)
+    qa, sa = ov.quant_act(f64(a))
+    qw, sw = ov.quant_weight(f64(w))
+    ref = ov.fp8_block_gemm(qa, sa, qw, sw, f64(bias), f64(res))
+    lds = (M + 3) // 4 * 4
+    sa_pad = np.zeros((sa.shape[0], lds), np.float32)
+    sa_pad[:, :M] = sa
+    dev = "cuda"
+    out = vitq.fp8_block_gemm(torch.from_numpy(qa).to(dev), torch.from_numpy(sa_pad).to(dev),
+                              torch.from_numpy(qw).to(dev), torch.from_numpy(sw).to(dev),
+                              bias.to(dev), res.to(dev))
+    got = f64(out)
+    assert_close(got, ref, what=f"gemm {M}x{N}x{K} bn{bn}")
+    # the promotion is fp32 against an fp64 oracle: nearly every bf16 output is identical
+    assert np.mean(got == ref) > 0.97
+
+
+def test_fp8_gemm_no_bias_no_residual(lib):
+    from quantized_vit_encoder_b200 import vitq
+    M, N, K = 200, 384, 640
+    a, w = bf16((M, K), 60, 2.0), bf16((N, K), 61, 0.05)
+    qa, sa = ov.quant_act(f64(a))
+    qw, sw = ov.quant_weight(f64(w))
+    ref = ov.fp8_block_gemm(qa, sa, qw, sw)
+    out = vitq.fp8_block_gemm(torch.from_numpy(qa).cuda(), torch.from_numpy(sa).cuda(),
+                              torch.from_numpy(qw).cuda(), torch.from_numpy(sw).cuda())
+    assert_close(f64(out), ref, what="gemm plain")
+
+
+# ----------------------------------------------------------------- positions and RoPE
+
+def test_positions_match_oracle(lib):
+    from quantized_vit_encoder_b200 import vitq
+    grids = [(54, 18), (46, 136), (24, 38), (32, 32), (36, 27), (1, 1)]
+    pos, cu = vitq.positions(grids)
+    pr, cr = ov.packed_positions(grids)
+    assert np.array_equal(pos.cpu().numpy(), pr)
+    assert np.array_equal(cu.cpu().numpy(), cr)
+
+
+def test_rope_table_and_apply(lib):
+    from quantized_vit_encoder_b200 import vitq
+    grids = [(46, 136), (36, 27)]
+    pos, _ = vitq.positions(grids)
+    cs = vitq.rope_table(pos)
+    pr, _ = ov.packed_positions(grids)
+    ang = ov.rope_angles(pr)
+    assert np.max(np.abs(cs.cpu().numpy()[:, :36] - np.cos(ang))) < 1e-6
+    assert np.max(np.abs(cs.cpu().numpy()[:, 36:] - np.sin(ang))) < 1e-6
+    n = pr.shape[0]
+    qkv = bf16((n, 3456), 70, 1.0)
+    got = vitq.rope2d_(qkv.cuda().clone(), cs)
+    ref = ov.apply_rope_qkv(f64(qkv), pr)
+    assert_close(f64(got), ref, what="rope")
+    assert np.array_equal(f64(got)[:, 2304:], f64(qkv)[:, 2304:])       # v untouched
+    # with VITQ_V_FP16 the q, k results are identical and v becomes its exact fp16 value
+    got16 = vitq.rope2d_(qkv.cuda().clone(), cs, flags=vitq.V_FP16)
+    assert torch.equal(got16[:, :2304], got[:, :2304])
+    v16 = got16[:, 2304:].contiguous().view(torch.float16).float().cpu().double().numpy()
+    assert np.array_equal(v16, f64(qkv)[:, 2304:])
+
+
+# ----------------------------------------------------------------- attention
+
+ATTN_CASES = [
+    [1], [127], [128], [129], [256], [300, 1, 77, 128], [972], [972, 6256, 912, 1024],
+]
+
+
+def _v_to_f16(qkv_dev):
+    """v part converted to fp16 in place (exact), as the block does before attention."""
+    t = qkv_dev.clone()
+    t[:, 2304:] = t[:, 2304:].float().half().view(torch.bfloat16)
+    return t
+
+
+@pytest.mark.parametrize("v16", [False, True], ids=["bf16v", "f16v"])
+@pytest.mark.parametrize("lens", ATTN_CASES, ids=lambda v: "-".join(map(str, v)))
+def test_attention_matches_oracle(lib, lens, v16):
+    from quantized_vit_encoder_b200 import vitq
+    n = sum(lens)
+    cu = wl.random_cu_seqlens(lens)
+    qkv = bf16((n, 3456), 80 + n, 1.0)
+    ref = ov.attention_varlen(f64(qkv), cu)
+    dq = _v_to_f16(qkv.cuda()) if v16 else qkv.cuda()
+    got = vitq.attention_varlen(dq, torch.tensor(cu, dtype=torch.int32, device="cuda"), max(lens),
+                                flags=vitq.V_FP16 if v16 else 0)
+    r, _ = assert_close(f64(got), ref, what=f"attention {lens}")
+    if v16 and n >= 128:
+        # fp16 P: the only remaining difference is the final bf16 rounding of O
+        assert r < 1.5e-3, r
+
+
+def test_attention_large_logits_rescale(lib):
+    """Scores spanning a wide range force the running-max rescale path."""
+    from quantized_vit_encoder_b200 import vitq
+    n = 700
+    g = torch.Generator().manual_seed(90)
+    qkv = torch.randn((n, 3456), generator=g)
+    qkv[:, :2304] *= torch.linspace(0.2, 4.0, n)[:, None]          # growing norms along the sequence
+    qkv = qkv.to(torch.bfloat16)
+    ref = ov.attention_varlen(f64(qkv), [0, n])
+    got = vitq.attention_varlen(qkv.cuda(), torch.tensor([0, n], dtype=torch.int32, device="cuda"), n)
+    assert_close(f64(got), ref, what="attention rescale")
+
+
+def test_attention_full_6256_sampled_rows(lib):
+    """Full 46x136 image: compare 256 sampled query rows of every head against the oracle."""
+    from quantized_vit_encoder_b200 import vitq
+    n = 6256
+    qkv = bf16((n, 3456), 95, 1.0)
+    got = f64(vitq.attention_varlen(qkv.cuda(), torch.tensor([0, n], dtype=torch.int32, device="cuda"), n))
+    rows = np.random.default_rng(1).choice(n, 256, replace=False)
+    t = f64(qkv).reshape(n, 3, 16, 72)
+    ref = np.zeros((256, 16, 72))
+    for h in range(16):
+        s = t[rows, 0, h] @ t[:, 1, h].T / math.sqrt(72)
+        s -= s.max(1, keepdims=True)
+        p = np.exp(s)
+        ref[:, h] = (p / p.sum(1, keepdims=True)) @ t[:, 2, h]
+    assert_close(got[rows], onum.bf16_round(ref.reshape(256, -1)), what="attention 6256 sampled")
