@@ -122,7 +122,8 @@ int fp8_block_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W
 int vit_rope_table(const int32_t* pos_hw, int n_tokens, float theta, float* cos_sin, void* stream);
 
 /* Flag for vit_rope2d / vit_attention_varlen: the v part of qkv is (made) fp16.
- * v comes out of a bf16 GEMM, so bf16 -> fp16 is exact (|v| < 65504), and the
+ * v comes out of a bf16 GEMM; bf16 -> fp16 (round to nearest) is exact for
+ * 2^-14 <= |v| < 65504 and off by at most 2^-25 below that, and the
  * attention then runs its P.V product with fp16 P (11 significant bits instead
  * of 8) at the same tensor-core rate. */
 #define VITQ_V_FP16 1

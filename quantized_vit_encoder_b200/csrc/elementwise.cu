@@ -304,8 +304,8 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int n, double
 // token's q and k heads (9 per head): x'_j = x_j c_j - x_(j+36) s_j,
 // x'_(j+36) = x_(j+36) c_j + x_j s_j; the partner elements of chunk cc live in
 // two neighbouring chunks A (elements 4..7) and B (elements 0..3).  Chunks
-// 288..431 are the v heads, converted to fp16 in place when v_to_f16 (bf16 ->
-// fp16 is exact for |v| < 65504).  All reads happen before the barrier and all
+// 288..431 are the v heads, converted to fp16 in place when v_to_f16 (round to
+// nearest: exact for 2^-14 <= |v| < 65504, within 2^-25 below).  All reads happen before the barrier and all
 // writes after it, so the in-place update never reads a rotated value.
 __global__ void __launch_bounds__(432) rope_apply_kernel(__nv_bfloat16* __restrict__ qkv,
                                                          const float* __restrict__ cs, int v_to_f16) {

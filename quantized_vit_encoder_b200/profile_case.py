@@ -1,0 +1,69 @@
+"""Run one stage of the block at the 46x136 (6256-patch) size a few times, for profilers.
+
+    python -m quantized_vit_encoder_b200.profile_case STAGE [--iters N]
+
+STAGE: attention | gemm_qkv | gemm_proj | gemm_fc1 | gemm_fc2 | ln_quant | gelu_quant | rope | block.
+Device memory stays below 0.5 GB; each iteration is one launch of the stage's
+kernel (block: the ten launches of one block).
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import vitq
+from . import workloads as wl
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("stage")
+    ap.add_argument("--iters", type=int, default=3)
+    a = ap.parse_args()
+    torch.cuda.set_device(0)
+    vitq.load()
+    W = wl.WORKLOADS["block_46x136"]
+    n = W.n_tokens
+    dev = "cuda"
+    x = wl.make_input(W).to(dev)
+    blk = vitq.DeviceBlock(wl.block_params(wl.block_seed(W, 0)), dev)
+    pos, cu = vitq.positions(list(W.grids), dev)
+    cs = vitq.rope_table(pos)
+    t = blk.t
+    if a.stage == "block":
+        ws = vitq.workspace(vitq.block_workspace_bytes(n), dev)
+        run = lambda: vitq.block_forward_(blk, x, cu, n, cs, ws)  # noqa: E731
+    elif a.stage == "attention":
+        qkv = wl.random_bf16((n, 3456), 1, 1.0).to(dev)
+        vitq.rope2d_(qkv, cs, flags=vitq.V_FP16)
+        out = torch.empty((n, 1152), dtype=torch.bfloat16, device=dev)
+        run = lambda: vitq.attention_varlen(qkv, cu, n, out=out, flags=vitq.V_FP16)  # noqa: E731
+    elif a.stage.startswith("gemm_"):
+        name = a.stage[5:]
+        w = t[name + "_w"]
+        K = w.shape[1]
+        act = wl.random_bf16((n, K), 2, 1.0).to(dev)
+        qa, sa = vitq.quant_act(act)
+        res = x if name in ("proj",) else (wl.random_bf16((n, 1152), 3).to(dev) if name == "fc2" else None)
+        out = torch.empty((n, w.shape[0]), dtype=torch.bfloat16, device=dev)
+        run = lambda: vitq.fp8_block_gemm(qa, sa, t[name + "_q"], t[name + "_s"], t[name + "_b"], res, out)  # noqa: E731
+    elif a.stage == "ln_quant":
+        run = lambda: vitq.ln_quant(x, t["norm1_w"], t["norm1_b"])  # noqa: E731
+    elif a.stage == "gelu_quant":
+        f = wl.random_bf16((n, 4304), 4, 1.0).to(dev)
+        run = lambda: vitq.gelu_quant(f)  # noqa: E731
+    elif a.stage == "rope":
+        qkv = wl.random_bf16((n, 3456), 5, 1.0).to(dev)
+        run = lambda: vitq.rope2d_(qkv, cs)  # noqa: E731
+    else:
+        raise SystemExit(f"unknown stage {a.stage}")
+    for _ in range(a.iters):
+        run()
+    torch.cuda.synchronize()
+    assert vitq.device_error() == 0
+    print(f"{a.stage}: {a.iters} iterations ok")
+
+
+if __name__ == "__main__":
+    main()
