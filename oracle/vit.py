@@ -29,7 +29,8 @@ design notes):
   * RoPE: inv_freq_i = theta**(-2i/36), i < 18; angles [row*f, col*f];
     rotate_half pairs (j, j+36); fp64, rounded to bf16.
   * attention: scale 1/sqrt(72), fp64 softmax, output rounded to bf16.
-  * GELU: tanh form in fp64, rounded to bf16 (blocks and mergers).
+  * GELU: tanh form, evaluated as x / (1 + exp(-2u)) in fp64 (no cancellation),
+    rounded to bf16 (blocks and mergers).
   * patch order: 2x2-block order for even grids (so the merger's 4
     neighbours are 4 consecutive rows), row-major otherwise.
   * merger: LayerNorm over the 4608 concatenated features, then
@@ -151,9 +152,16 @@ def layernorm(x, gamma, beta, eps: float = 1e-6) -> np.ndarray:
 
 
 def gelu_tanh_f64(x) -> np.ndarray:
-    """0.5 x (1 + tanh(sqrt(2/pi) (x + 0.044715 x^3))) in fp64, not rounded."""
+    """GELU(tanh) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3), in fp64, not rounded.
+
+    Evaluated as x / (1 + exp(-2u)), which equals 0.5 x (1 + tanh(u)) exactly
+    (1 + tanh(u) = 2 / (1 + exp(-2u))) but does not cancel for u << 0, where
+    1 + tanh(u) in fp64 loses all its digits (u < -19, x < -5.6).
+    """
     x = np.asarray(x, np.float64)
-    return 0.5 * x * (1.0 + np.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+    u = math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)
+    with np.errstate(over="ignore"):
+        return x / (1.0 + np.exp(-2.0 * u))
 
 
 def gelu_tanh(x) -> np.ndarray:

@@ -6,15 +6,19 @@
 // with cu_seqlens): O = softmax(Q K^T * scale) V per segment and head.
 //
 // Design (B200):
-//   * one CTA per (segment, head, 128-query tile); 6 warps: TMA producer, MMA
-//     issuer, 4 softmax warps (one thread per query row = one TMEM lane);
+//   * one CTA per (segment, head, 256 queries = two 128-row Q tiles); 12 warps:
+//     TMA producer, one MMA issuer per Q tile, and one softmax warpgroup per Q
+//     tile (thread = query row = TMEM lane).  S_x(j+1) is computed while the
+//     softmax of S_x(j) runs (the softmax frees S_x once it holds it in
+//     registers), and the two tiles interleave on the tensor core;
+//   * the softmax exponentials run on MUFU ex2; a share can move to a polynomial
+//     on the FMA pipe (kPolyEvery) to balance the two pipes;
 //   * Q, K, V are read straight from the packed qkv activation [n, 3, 16, 72]
 //     through 3D TMA maps (d, slot, token).  head_dim 72 is padded to 80 by
 //     the tensor map itself: d 0..63 land in a 128B-swizzled tile and d 64..79
 //     in a 32B-swizzled tile, and d >= 72 lies outside the map so TMA fills
 //     zeros.  The padding never exists in HBM;
-//   * S = Q K^T runs as 5 tcgen05.mma (K = 16 each) into one of two TMEM
-//     buffers, so the next tile's scores overlap this tile's softmax;
+//   * S = Q K^T runs as 5 tcgen05.mma (K = 16 each) into the tile's TMEM S buffer;
 //   * the softmax warps keep a running max in the log2 domain and rescale O
 //     (in TMEM) only when the max grows by more than 8, write P as bf16 into a
 //     128B-swizzled shared tile, and the MMA warp accumulates O += P V with V
@@ -28,15 +32,32 @@
 namespace vitq {
 namespace {
 
-constexpr int kBM = 128, kBN = 128, kStages = 3;
-constexpr int kQLo = 0, kQHi = 16384;
-constexpr int kKV0 = 20480, kKVStride = 40960;
+constexpr int kBM = 128, kBN = 128, kStages = 3, kQTiles = 2;
+// Shared memory: Q tiles (A, B), a ring of K/V stages, the P tiles (A, B).
+constexpr int kQBytes = 20480;                          // 128 x 64 (SW128) + 128 x 16 (SW32), bf16
+constexpr int kQLo = 0, kQHi = 16384;                   // offsets inside a Q tile
+constexpr int kKV0 = kQTiles * kQBytes, kKVStride = 40960;
 constexpr int kKLo = 0, kKHi = 16384, kVLo = 20480, kVHi = 36864;
-constexpr int kP = kKV0 + kStages * kKVStride;          // two 64-key atoms of 16 KB
-constexpr int kBar = kP + 32768;
-constexpr int kNumBars = 1 + 2 * kStages + 2 + 1 + 1;
+constexpr int kP0 = kKV0 + kStages * kKVStride;         // P tile X: two 64-key atoms of 16 KB
+constexpr int kPBytes = 32768;
+constexpr int kBar = kP0 + kQTiles * kPBytes;
+// barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], s_free[2]
+constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles;
 constexpr size_t kAttnSmem = 1024 + kBar + kNumBars * 8 + 16;
-constexpr uint32_t kTmemS = 0, kTmemO = 256;
+static_assert(kAttnSmem <= 232448, "shared memory budget");
+// TMEM columns: S_A 0..127, S_B 128..255, O_A 256..335, O_B 384..463.
+__device__ __forceinline__ uint32_t tmem_s(int x) { return (uint32_t)x * 128u; }
+__device__ __forceinline__ uint32_t tmem_o(int x) { return 256u + (uint32_t)x * 128u; }
+// Warpgroup 0: warp 0 TMA producer, warps 1 and 2 MMA issuers for Q tiles A
+// and B (warp 3 idle); warpgroups 1 and 2: softmax of Q tiles A and B.
+constexpr int kThreads = 128 * (1 + kQTiles);
+// Share of the softmax exponentials moved from MUFU to the FMA-pipe polynomial:
+// one pair in kPolyEvery (0 = none).  MUFU ex2 runs at 16 per clock per SM.
+#ifndef VITQ_ATTN_POLY_EVERY
+#define VITQ_ATTN_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = VITQ_ATTN_POLY_EVERY;
+constexpr int kPolyMod = kPolyEvery > 0 ? kPolyEvery : 1;
 
 struct AttnArgs {
   const int32_t* cu;
@@ -45,6 +66,18 @@ struct AttnArgs {
   float scale_log2;
 };
 
+// K/V tiles are visited starting at a per-CTA offset so that the CTAs of one
+// head, which run at the same time, read different K/V tiles (online softmax
+// does not depend on the order).  The offset depends only on the Q-tile index
+// within its segment, so a segment gives the same result packed or alone.
+#ifndef VITQ_ATTN_STAGGER
+#define VITQ_ATTN_STAGGER 1
+#endif
+__device__ __forceinline__ int kv_tile(int j, int off, int n_kv) {
+  const int t = j + off;
+  return t >= n_kv ? t - n_kv : t;
+}
+
 struct AttnSmem {
   uint8_t* base;
   __device__ uint32_t at(int off) const { return smem_u32(base + off); }
@@ -52,14 +85,17 @@ struct AttnSmem {
   __device__ uint32_t q_full() const { return smem_u32(bar(0)); }
   __device__ uint32_t kv_full(int s) const { return smem_u32(bar(1 + s)); }
   __device__ uint32_t kv_empty(int s) const { return smem_u32(bar(1 + kStages + s)); }
-  __device__ uint32_t s_full(int b) const { return smem_u32(bar(1 + 2 * kStages + b)); }
-  __device__ uint32_t p_full() const { return smem_u32(bar(3 + 2 * kStages)); }
-  __device__ uint32_t pv_done() const { return smem_u32(bar(4 + 2 * kStages)); }
+  __device__ uint32_t s_full(int x) const { return smem_u32(bar(1 + 2 * kStages + x)); }
+  __device__ uint32_t p_full(int x) const { return smem_u32(bar(1 + 2 * kStages + kQTiles + x)); }
+  __device__ uint32_t pv_done(int x) const { return smem_u32(bar(1 + 2 * kStages + 2 * kQTiles + x)); }
+  __device__ uint32_t s_free(int x) const { return smem_u32(bar(1 + 2 * kStages + 3 * kQTiles + x)); }
   __device__ uint32_t* tmem_holder() const { return reinterpret_cast<uint32_t*>(bar(kNumBars)); }
   __device__ volatile int* abort_flag() const {
     return reinterpret_cast<volatile int*>(tmem_holder() + 1);
   }
+  __device__ uint32_t q(int x, int part) const { return at(x * kQBytes + part); }
   __device__ uint32_t kv(int s, int part) const { return at(kKV0 + s * kKVStride + part); }
+  __device__ uint32_t p(int x) const { return at(kP0 + x * kPBytes); }
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -68,17 +104,65 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 2^x on the FMA/ALU pipes for a pair of values (Cody-Waite split x = n + f,
+// |f| <= 1/2, then a degree-3 polynomial fitted to 2^f on [-1/2, 1/2]: max
+// relative error 7.5e-5, below the fp16 rounding of P).  n is read from the low
+// bits of x + 1.5*2^23 and added to the exponent field; x is clamped at -125
+// (2^-125 is 0 once P is rounded).
+__device__ __forceinline__ uint64_t f2pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 f2unpack(uint64_t v) {
+  float2 f;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+  return f;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// ex2_poly on a pair of values with packed fp32 arithmetic.
+__device__ __forceinline__ float2 ex2_poly2(float x0, float x1) {
+  const uint64_t magic = f2pack(12582912.0f, 12582912.0f), nmagic = f2pack(-12582912.0f, -12582912.0f);
+  const uint64_t x = f2pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t j = fadd2(x, magic);
+  const uint64_t f = ffma2(fadd2(j, nmagic), f2pack(-1.0f, -1.0f), x);
+  uint64_t p = ffma2(f2pack(0.0551716648f, 0.0551716648f), f, f2pack(0.2426111251f, 0.2426111251f));
+  p = ffma2(p, f, f2pack(0.6932609677f, 0.6932609677f));
+  p = ffma2(p, f, f2pack(0.9999280572f, 0.9999280572f));
+  const float2 pp = f2unpack(p), jj = f2unpack(j);
+  return make_float2(__int_as_float(__float_as_int(pp.x) + (__float_as_int(jj.x) << 23)),
+                     __int_as_float(__float_as_int(pp.y) + (__float_as_int(jj.y) << 23)));
+}
+
+
+
 __device__ void attn_producer(const AttnSmem& sm, const CUtensorMap* tlo, const CUtensorMap* thi,
-                              int head, int q_row, int kv_row0, int n_kv) {
-  mbar_arrive_expect_tx(sm.q_full(), 20480);
-  tma_load_3d(sm.at(kQLo), tlo, 0, head, q_row, sm.q_full());
-  tma_load_3d(sm.at(kQHi), thi, 64, head, q_row, sm.q_full());
+                              int head, int q_row, int n_q, int kv_row0, int n_kv, int off) {
+  mbar_arrive_expect_tx(sm.q_full(), kQBytes * n_q);
+  for (int x = 0; x < n_q; ++x) {
+    tma_load_3d(sm.q(x, kQLo), tlo, 0, head, q_row + x * kBM, sm.q_full());
+    tma_load_3d(sm.q(x, kQHi), thi, 64, head, q_row + x * kBM, sm.q_full());
+  }
   for (int j = 0; j < n_kv; ++j) {
     const int s = j % kStages;
     const uint32_t ph = (uint32_t)(j / kStages) & 1u;
     if (!mbar_wait(sm.kv_empty(s), ph ^ 1u, sm.abort_flag())) return;
     mbar_arrive_expect_tx(sm.kv_full(s), 40960);
-    const int row = kv_row0 + j * kBN;
+    const int row = kv_row0 + kv_tile(j, off, n_kv) * kBN;
     tma_load_3d(sm.kv(s, kKLo), tlo, 0, 16 + head, row, sm.kv_full(s));
     tma_load_3d(sm.kv(s, kKHi), thi, 64, 16 + head, row, sm.kv_full(s));
     tma_load_3d(sm.kv(s, kVLo), tlo, 0, 32 + head, row, sm.kv_full(s));
@@ -86,50 +170,64 @@ __device__ void attn_producer(const AttnSmem& sm, const CUtensorMap* tlo, const 
   }
 }
 
-__device__ bool attn_issue_s(const AttnSmem& sm, uint32_t tmem, int j) {
+// S_x = Q_x K_j^T (5 MMAs of K = 16 over the padded head_dim 80) into S buffer x.
+__device__ bool attn_issue_s(const AttnSmem& sm, uint32_t tmem, int x, int j) {
   constexpr uint32_t idesc = make_idesc(1, 1, 0, 0, 128, 128);
   const int s = j % kStages;
   if (!mbar_wait(sm.kv_full(s), (uint32_t)(j / kStages) & 1u, sm.abort_flag())) return false;
   tc_fence_after();
-  const uint32_t d = tmem + kTmemS + (uint32_t)(j & 1) * 128;
-  const uint32_t qlo = sm.at(kQLo), klo = sm.kv(s, kKLo);
+  const uint32_t d = tmem + tmem_s(x);
+  const uint32_t qlo = sm.q(x, kQLo), klo = sm.kv(s, kKLo);
 #pragma unroll
   for (int k = 0; k < 4; ++k)
     mma_bf16_ss(d, make_smem_desc(qlo + 32 * k, 16, 1024, kSwizzle128B),
                 make_smem_desc(klo + 32 * k, 16, 1024, kSwizzle128B), idesc, k > 0 ? 1u : 0u);
-  mma_bf16_ss(d, make_smem_desc(sm.at(kQHi), 16, 256, kSwizzle32B),
+  mma_bf16_ss(d, make_smem_desc(sm.q(x, kQHi), 16, 256, kSwizzle32B),
               make_smem_desc(sm.kv(s, kKHi), 16, 256, kSwizzle32B), idesc, 1u);
-  tc_commit(sm.s_full(j & 1));
+  tc_commit(sm.s_full(x));
   return true;
 }
 
+// O_x += P_x V_j: P from shared memory (K-major), V MN-major; N = 64 + 16.
 template <bool kVF16>
-__device__ void attn_mma(const AttnSmem& sm, uint32_t tmem, int n_kv) {
-  // P.V operands: fp16 (format 0) when v was converted to fp16, else bf16 (format 1).
+__device__ bool attn_issue_pv(const AttnSmem& sm, uint32_t tmem, int x, int j) {
   constexpr uint32_t fmt = kVF16 ? 0u : 1u;
   constexpr uint32_t idesc_lo = make_idesc(fmt, fmt, 0, 1, 128, 64);
   constexpr uint32_t idesc_hi = make_idesc(fmt, fmt, 0, 1, 128, 16);
-  if (!mbar_wait(sm.q_full(), 0, sm.abort_flag())) return;
-  if (!attn_issue_s(sm, tmem, 0)) return;
-  if (n_kv > 1 && !attn_issue_s(sm, tmem, 1)) return;
-  const uint32_t p0 = sm.at(kP);
-  for (int j = 0; j < n_kv; ++j) {
-    if (!mbar_wait(sm.p_full(), (uint32_t)j & 1u, sm.abort_flag())) return;
-    tc_fence_after();
-    const int s = j % kStages;
-    const uint32_t vlo = sm.kv(s, kVLo), vhi = sm.kv(s, kVHi);
+  if (!mbar_wait(sm.p_full(x), (uint32_t)j & 1u, sm.abort_flag())) return false;
+  tc_fence_after();
+  const int s = j % kStages;
+  const uint32_t vlo = sm.kv(s, kVLo), vhi = sm.kv(s, kVHi), p0 = sm.p(x);
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint64_t ad = make_smem_desc(p0 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B);
-      const uint32_t acc = (j > 0 || k > 0) ? 1u : 0u;
-      mma_bf16_ss(tmem + kTmemO, ad, make_smem_desc(vlo + k * 2048, 16384, 1024, kSwizzle128B), idesc_lo,
-                  acc);
-      mma_bf16_ss(tmem + kTmemO + 64, ad, make_smem_desc(vhi + k * 512, 4096, 256, kSwizzle32B), idesc_hi,
-                  acc);
+  for (int k = 0; k < 8; ++k) {
+    const uint64_t ad = make_smem_desc(p0 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B);
+    const uint32_t acc = (j > 0 || k > 0) ? 1u : 0u;
+    mma_bf16_ss(tmem + tmem_o(x), ad, make_smem_desc(vlo + k * 2048, 16384, 1024, kSwizzle128B), idesc_lo, acc);
+    mma_bf16_ss(tmem + tmem_o(x) + 64, ad, make_smem_desc(vhi + k * 512, 4096, 256, kSwizzle32B), idesc_hi, acc);
+  }
+  tc_commit(sm.pv_done(x));
+  return true;
+}
+
+// Tensor-core work of Q tile x, issued by its own thread.  S_x(j+1) is issued as
+// soon as the softmax has moved S_x(j) into registers (s_free), so it overlaps
+// that softmax; P_x(j).V_j follows when P_x(j) is in shared memory.  The two
+// tiles' threads interleave on the tensor core; a K/V stage is released when
+// both tiles' P.V of that stage have completed (kv_empty counts one commit per tile).
+template <bool kVF16>
+__device__ void attn_mma(const AttnSmem& sm, uint32_t tmem, int x, int n_kv) {
+  if (!mbar_wait(sm.q_full(), 0, sm.abort_flag())) return;
+  if (!attn_issue_s(sm, tmem, x, 0)) return;
+  for (int j = 0; j < n_kv; ++j) {
+    if (j + 1 < n_kv) {
+      if (!mbar_wait(sm.s_free(x), (uint32_t)j & 1u, sm.abort_flag())) return;
+      tc_fence_after();
+      if (!attn_issue_s(sm, tmem, x, j + 1)) return;
+      VITQ_TRACE_EV(10 + x);   // mma: S issued
     }
-    tc_commit(sm.pv_done());
-    tc_commit(sm.kv_empty(s));
-    if (j + 2 < n_kv && !attn_issue_s(sm, tmem, j + 2)) return;
+    if (!attn_issue_pv<kVF16>(sm, tmem, x, j)) return;
+    VITQ_TRACE_EV(12 + x);     // mma: P.V issued
+    tc_commit(sm.kv_empty(j % kStages));
   }
 }
 
@@ -141,76 +239,75 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi, bool f16) {
   return pack_bf16x2(lo, hi);
 }
 
-__device__ __forceinline__ float2 unpack_p(uint32_t u, bool f16) {
-  if (f16) {
-    __half2 h = *reinterpret_cast<__half2*>(&u);
-    return __half22float2(h);
-  }
-  return unpack_bf16x2(u);
-}
-
+// One warpgroup per Q tile; thread = query row = TMEM lane.  S is read from
+// TMEM twice (row max, then exponentials), 64 columns at a time, so a thread
+// holds at most 64 scores in registers.
 template <bool kVF16>
-__device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& g, int head, int seq_start,
-                             int seq_len, int q0, int n_kv) {
+__device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& g, int x, int head,
+                             int seq_start, int seq_len, int q0, int n_kv, int off) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;
   const int r = quad * 32 + lane;
   const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-  uint8_t* pbase = sm.base + kP;
+  const uint32_t s_addr = tmem + lane_addr + tmem_s(x), o_addr = tmem + lane_addr + tmem_o(x);
+  uint8_t* pbase = sm.base + kP0 + x * kPBytes;
   float m_run = -INFINITY, l_run = 0.f;
   for (int j = 0; j < n_kv; ++j) {
-    bool ok = mbar_wait(sm.s_full(j & 1), (uint32_t)(j >> 1) & 1u, sm.abort_flag());
+    bool ok = mbar_wait(sm.s_full(x), (uint32_t)j & 1u, sm.abort_flag());
     if (!__all_sync(0xffffffffu, ok)) return;
+    if (lane == 0 && quad == 0) VITQ_TRACE_EV(20 + x);   // softmax: S ready
     tc_fence_after();
-    float sv[128];
+    const int valid = seq_len - kv_tile(j, off, n_kv) * kBN;   // keys of this tile inside the segment
+    // one TMEM round trip: all 128 scores of the row, then S_x is free for S_x(j+1)
+    uint32_t su[4][32];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      uint32_t u[32];
-      tmem_ld32(tmem + lane_addr + kTmemS + (uint32_t)(j & 1) * 128 + c * 32, u);
-      tmem_wait_ld();
-#pragma unroll
-      for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(u[i]);
-    }
-    const int valid = seq_len - j * kBN;
+    for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, su[c]);
+    tmem_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.s_free(x));
     if (valid < kBN) {
 #pragma unroll
       for (int i = 0; i < 128; ++i)
-        if (i >= valid) sv[i] = -INFINITY;
+        if (i >= valid) su[i >> 5][i & 31] = 0xFF800000u;   // -inf
     }
-    float mx = -INFINITY;
+    // row max: 8 independent chains of 3-input max, then a tree
+    float mp[8];
 #pragma unroll
-    for (int i = 0; i < 128; ++i) mx = fmaxf(mx, sv[i]);
-    mx *= g.scale_log2;
+    for (int k = 0; k < 8; ++k) mp[k] = __uint_as_float(su[0][k]);
+#pragma unroll
+    for (int i = 8; i < 128; i += 16)
+#pragma unroll
+      for (int k = 0; k < 8; ++k)
+        mp[k] = fmax3(mp[k], __uint_as_float(su[(i + k) >> 5][(i + k) & 31]),
+                      __uint_as_float(su[(i + 8 + k) >> 5][(i + 8 + k) & 31]));
+    const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) *
+                     g.scale_log2;
     if (j > 0) {
-      ok = mbar_wait(sm.pv_done(), (uint32_t)(j - 1) & 1u, sm.abort_flag());
+      ok = mbar_wait(sm.pv_done(x), (uint32_t)(j - 1) & 1u, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
       tc_fence_after();
     }
+    if (lane == 0 && quad == 0) VITQ_TRACE_EV(22 + x);   // softmax: max known, O stable
+    // new running max: it changes only when the tile max exceeds it by more than 8
+    // (so P <= 2^8), and the decision is warp-uniform because the O rescale uses
+    // warp-collective tcgen05.ld/st (rows that keep their max get alpha = 1).
+    float alpha = 1.f;
+    bool rescale = false;
     if (j == 0) {
       m_run = mx;
     } else {
-      // tcgen05.ld/st are warp-collective: the whole warp rescales when any of
-      // its rows needs it, with alpha = 1 for rows that keep their max.
       const bool need = mx > m_run + 8.f;
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_new = need ? mx : m_run;
-        const float alpha = ex2(m_run - m_new);
-#pragma unroll
-        for (int c = 0; c < 5; ++c) {
-          uint32_t u[16];
-          tmem_ld16(tmem + lane_addr + kTmemO + c * 16, u);
-          tmem_wait_ld();
-#pragma unroll
-          for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
-          tmem_st16(tmem + lane_addr + kTmemO + c * 16, u);
-        }
-        tmem_wait_st();
-        l_run *= alpha;
-        m_run = m_new;
+      rescale = __any_sync(0xffffffffu, need);
+      if (need) {
+        alpha = ex2(m_run - mx);
+        m_run = mx;
       }
     }
-    // P = 2^(s * scale_log2 - m_run), rounded to the P.V operand type, into the swizzled P tile.
-    float lsum = 0.f;
+    // P = 2^(s * scale_log2 - m_run), rounded to the P.V operand type, into the swizzled
+    // P tile (64-key atom a holds keys 64a..64a+63); 8 fp32 partial row sums.
+    const uint64_t sc2 = f2pack(g.scale_log2, g.scale_log2), nm2 = f2pack(-m_run, -m_run);
+    uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int a = 0; a < 2; ++a) {
 #pragma unroll
@@ -219,60 +316,86 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int k0 = a * 64 + c * 8 + 2 * i;
-          const float p0 = ex2(fmaf(sv[k0], g.scale_log2, -m_run));
-          const float p1 = ex2(fmaf(sv[k0 + 1], g.scale_log2, -m_run));
-          w[i] = pack_p(p0, p1, kVF16);
-          const float2 pr = unpack_p(w[i], kVF16);
-          lsum += pr.x + pr.y;
+          const float2 t = f2unpack(ffma2(f2pack(__uint_as_float(su[k0 >> 5][k0 & 31]),
+                                                 __uint_as_float(su[(k0 + 1) >> 5][(k0 + 1) & 31])),
+                                          sc2, nm2));
+          // every kPolyEvery-th pair runs the FMA-pipe polynomial, the rest MUFU ex2
+          float2 p;
+          if (kPolyEvery > 0 && (i % kPolyMod) == kPolyMod - 1) {
+            p = ex2_poly2(t.x, t.y);
+          } else {
+            p.x = ex2(t.x);
+            p.y = ex2(t.y);
+          }
+          w[i] = pack_p(p.x, p.y, kVF16);
+          ls[i] = fadd2(ls[i], f2pack(p.x, p.y));
         }
         uint8_t* dst = pbase + a * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
         *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
-    l_run += lsum;
+    if (rescale) {
+      // O (complete up to P.V(j-1)) to the new max; done after P so the scores are dead
+      uint32_t u[5][16];
+#pragma unroll
+      for (int c = 0; c < 5; ++c) tmem_ld16(o_addr + c * 16, u[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 5; ++c) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) u[c][i] = __float_as_uint(__uint_as_float(u[c][i]) * alpha);
+        tmem_st16(o_addr + c * 16, u[c]);
+      }
+      tmem_wait_st();
+    }
+    {
+      const float2 l0 = f2unpack(fadd2(ls[0], ls[1])), l1 = f2unpack(fadd2(ls[2], ls[3]));
+      l_run = l_run * alpha + ((l0.x + l0.y) + (l1.x + l1.y));
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(sm.p_full());
+    if (lane == 0 && quad == 0) VITQ_TRACE_EV(24 + x);   // softmax: P written
+    if (lane == 0) mbar_arrive(sm.p_full(x));
   }
-  bool ok = mbar_wait(sm.pv_done(), (uint32_t)(n_kv - 1) & 1u, sm.abort_flag());
+  bool ok = mbar_wait(sm.pv_done(x), (uint32_t)(n_kv - 1) & 1u, sm.abort_flag());
   if (!__all_sync(0xffffffffu, ok)) return;
   tc_fence_after();
-  float o[80];
+  // O / l in 16-column chunks (columns 72..79 are the zero padding and are not stored)
+  const bool row_ok = q0 + r < seq_len && seq_start + q0 + r < g.n_tokens;
+  const float inv = 1.0f / l_run;
+  __nv_bfloat16* dst = g.out + (size_t)(seq_start + q0 + r) * 1152 + head * 72;
+  uint32_t u[5][16];
 #pragma unroll
-  for (int c = 0; c < 5; ++c) {
-    uint32_t u[16];
-    tmem_ld16(tmem + lane_addr + kTmemO + c * 16, u);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 16; ++i) o[c * 16 + i] = __uint_as_float(u[i]);
-  }
-  if (q0 + r < seq_len && seq_start + q0 + r < g.n_tokens) {
-    const float inv = 1.0f / l_run;
-    __nv_bfloat16* dst = g.out + (size_t)(seq_start + q0 + r) * 1152 + head * 72;
+  for (int c = 0; c < 5; ++c) tmem_ld16(o_addr + c * 16, u[c]);
+  tmem_wait_ld();
+  if (row_ok) {
 #pragma unroll
     for (int c8 = 0; c8 < 9; ++c8) {
-      uint4 u;
-      u.x = pack_bf16x2(o[c8 * 8 + 0] * inv, o[c8 * 8 + 1] * inv);
-      u.y = pack_bf16x2(o[c8 * 8 + 2] * inv, o[c8 * 8 + 3] * inv);
-      u.z = pack_bf16x2(o[c8 * 8 + 4] * inv, o[c8 * 8 + 5] * inv);
-      u.w = pack_bf16x2(o[c8 * 8 + 6] * inv, o[c8 * 8 + 7] * inv);
-      *reinterpret_cast<uint4*>(dst + c8 * 8) = u;
+      const int c = c8 >> 1, h = c8 & 1;
+      uint4 v;
+      v.x = pack_bf16x2(__uint_as_float(u[c][h * 8 + 0]) * inv, __uint_as_float(u[c][h * 8 + 1]) * inv);
+      v.y = pack_bf16x2(__uint_as_float(u[c][h * 8 + 2]) * inv, __uint_as_float(u[c][h * 8 + 3]) * inv);
+      v.z = pack_bf16x2(__uint_as_float(u[c][h * 8 + 4]) * inv, __uint_as_float(u[c][h * 8 + 5]) * inv);
+      v.w = pack_bf16x2(__uint_as_float(u[c][h * 8 + 6]) * inv, __uint_as_float(u[c][h * 8 + 7]) * inv);
+      *reinterpret_cast<uint4*>(dst + c8 * 8) = v;
     }
   }
 }
 
 template <bool kVF16>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tlo, const __grid_constant__ CUtensorMap thi,
                 const AttnArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  const int qt = blockIdx.x, head = blockIdx.y, seq = blockIdx.z;
+  const int head = blockIdx.y, seq = blockIdx.z;
   const int seq_start = args.cu[seq];
   const int seq_len = args.cu[seq + 1] - seq_start;
-  const int q0 = qt * kBM;
+  const int q0 = blockIdx.x * kBM * kQTiles;
   if (q0 >= seq_len) return;
+  const int n_q = (seq_len - q0) > kBM ? kQTiles : 1;   // Q tiles of this CTA that hold rows
   const int n_kv = (seq_len + kBN - 1) / kBN;
+  const int off = VITQ_ATTN_STAGGER ? (int)((blockIdx.x * 7u) % (unsigned)n_kv) : 0;
   AttnSmem sm;
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -280,12 +403,14 @@ __global__ void __launch_bounds__(192, 1)
     mbar_init(sm.q_full(), 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(sm.kv_full(s), 1);
-      mbar_init(sm.kv_empty(s), 1);
+      mbar_init(sm.kv_empty(s), (uint32_t)n_q);       // one commit per active Q tile
     }
-    mbar_init(sm.s_full(0), 1);
-    mbar_init(sm.s_full(1), 1);
-    mbar_init(sm.p_full(), 4);
-    mbar_init(sm.pv_done(), 1);
+    for (int x = 0; x < kQTiles; ++x) {
+      mbar_init(sm.s_full(x), 1);
+      mbar_init(sm.p_full(x), 4);
+      mbar_init(sm.pv_done(x), 1);
+      mbar_init(sm.s_free(x), 4);
+    }
     *sm.abort_flag() = 0;
     fence_barrier_init();
   }
@@ -297,16 +422,17 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *sm.tmem_holder();
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < 4) {
+    if (warp == 0 && lane == 0) {
       prefetch_tensormap(&tlo);
       prefetch_tensormap(&thi);
-      attn_producer(sm, &tlo, &thi, head, seq_start + q0, seq_start, n_kv);
+      attn_producer(sm, &tlo, &thi, head, seq_start + q0, n_q, seq_start, n_kv, off);
+    } else if ((warp == 1 || warp == 2) && lane == 0 && warp - 1 < n_q) {
+      attn_mma<kVF16>(sm, tmem, warp - 1, n_kv);
     }
-  } else if (warp == 1) {
-    if (lane == 0) attn_mma<kVF16>(sm, tmem, n_kv);
   } else {
-    attn_softmax<kVF16>(sm, tmem, args, head, seq_start, seq_len, q0, n_kv);
+    const int x = (warp >> 2) - 1;
+    if (x < n_q) attn_softmax<kVF16>(sm, tmem, args, x, head, seq_start, seq_len, q0 + x * kBM, n_kv, off);
   }
   tc_fence_before();
   __syncthreads();
@@ -332,8 +458,8 @@ cudaError_t launch_attention(const __nv_bfloat16* qkv, int n_tokens, const int32
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
   if (e != cudaSuccess) return e;
   AttnArgs a{cu, out, n_tokens, scale * 1.4426950408889634f};
-  dim3 grid((max_seqlen + kBM - 1) / kBM, 16, n_seqs);
-  kern<<<grid, 192, kAttnSmem, st>>>(tlo, thi, a);
+  dim3 grid((max_seqlen + kBM * kQTiles - 1) / (kBM * kQTiles), 16, n_seqs);
+  kern<<<grid, kThreads, kAttnSmem, st>>>(tlo, thi, a);
   return cudaGetLastError();
 }
 

@@ -34,13 +34,19 @@ __device__ __forceinline__ float e4m3_quotient(float y, float s, float r) {
 }
 
 // Quantise 8 consecutive values of one 128-column group given the group scale.
+// A scale below the fp32 normal range (amax < 448 * 2^-126) has no finite
+// reciprocal; those groups always divide exactly.
 __device__ __forceinline__ uint2 quant8(const float (&v)[8], float s) {
   uint32_t c[4] = {0u, 0u, 0u, 0u};
-  if (s > 0.f) {
+  if (s >= 1.17549435e-38f) {
     const float r = __frcp_rn(s);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
       c[i] = cvt_e4m3x2(e4m3_quotient(v[2 * i], s, r), e4m3_quotient(v[2 * i + 1], s, r));
+  } else if (s > 0.f) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      c[i] = cvt_e4m3x2(__fdiv_rn(v[2 * i], s), __fdiv_rn(v[2 * i + 1], s));
   }
   return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
 }
@@ -197,10 +203,11 @@ __global__ void ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
 
 // ------------------------------------------------------------- GELU + quant
 // GELU(tanh) = 0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)), u = sqrt(2/pi)(x + 0.044715 x^3).
-// The fp32 sigmoid form (hardware exp2 and reciprocal) has no cancellation and a
-// relative error below 2^-16 for x >= -9; when its result lies within that bound
-// of a bf16 rounding midpoint, or x < -9, the value is recomputed in fp64 in the
-// tanh form, so the bf16 result is the rounding of the fp64 GELU.
+// The fp32 sigmoid form (hardware exp2 and reciprocal) has no cancellation; its
+// relative error is below 2^-21 (|u| + 2) (measured against fp64 over x in
+// [-12, 9]).  When the result lies within 2^-20 (|u| + 4) |g| of a bf16 rounding
+// midpoint (or is too small for that test) it is recomputed in fp64, so the
+// bf16 result is the rounding of the fp64 value x / (1 + exp(-2u)).
 
 __device__ __forceinline__ float gelu_tanh_bf16(float x) {
   const float u = x * fmaf(0.035677408136300125f, x * x, 0.7978845608028654f);
@@ -209,10 +216,11 @@ __device__ __forceinline__ float gelu_tanh_bf16(float x) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.0f + e));
   const float g = x * rc;
   float gr, dist;
-  if (x < -9.0f || !bf16_round_margin(g, &gr, &dist) || dist <= fabsf(g) * 1.52587890625e-05f) {  // 2^-16
+  const float err = fabsf(g) * (fabsf(u) + 4.0f) * 9.5367431640625e-07f;  // 2^-20
+  if (!bf16_round_margin(g, &gr, &dist) || dist <= err) {
     const double xd = (double)x;
     const double ud = 0.79788456080286535588 * (xd + 0.044715 * xd * xd * xd);
-    gr = __bfloat162float(__double2bfloat16(0.5 * xd * (1.0 + tanh(ud))));
+    gr = __bfloat162float(__double2bfloat16(xd / (1.0 + exp(-2.0 * ud))));
   }
   return gr;
 }

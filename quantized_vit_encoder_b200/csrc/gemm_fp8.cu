@@ -23,6 +23,9 @@
 namespace vitq {
 namespace {
 
+// BN = 128: 6 warps (TMA, MMA, 4 epilogue warps).  BN = 256: 12 warps
+// (warpgroup 0 = TMA, MMA and two idle warps, which give registers away with
+// setmaxnreg; warpgroups 1-2 = 8 epilogue warps, one per 128 columns x 32 rows).
 template <int BN>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 128;
@@ -32,10 +35,14 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NBUF = 512 / BN;
   static constexpr int EPI_WARPS = BN / 32;
-  static constexpr int THREADS = 64 + BN;
+  static constexpr int EPI_WARP0 = BN == 256 ? 4 : 2;
+  static constexpr int THREADS = BN == 256 ? 384 : 192;
+  static constexpr bool SPLIT_REGS = BN == 256;
+  static constexpr int MIN_LAUNCH_REGS = 168;   // 384 x 168 >= 128 x 56 + 256 x 224 (BN = 256)
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF) * 8 + 16;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
 };
+static_assert(384 * GemmCfg<256>::MIN_LAUNCH_REGS >= 128 * 56 + 256 * 224, "register split");
 
 struct GemmArgs {
   const float* sA;
@@ -72,17 +79,32 @@ struct GemmSmem {
   }
 };
 
+// Tile t -> (m, n): m = t % tiles_m, n = (t / tiles_m + m) % tiles_n.  A bijection
+// on the tile grid in which the CTAs running at the same time read different W
+// tiles (and each A tile is read by few of them), spreading the L2 traffic.
+#ifndef VITQ_GEMM_DIAG
+#define VITQ_GEMM_DIAG 1
+#endif
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int& m, int& n) {
+  m = tile % tiles_m;
+  const int q = tile / tiles_m;
+  n = VITQ_GEMM_DIAG ? (q + m) % tiles_n : q;
+}
+
 template <int BN>
 __device__ void gemm_producer(const GemmSmem<BN>& sm, const CUtensorMap* tmA, const CUtensorMap* tmB,
-                              int tiles_m, int num_tiles, int nkb) {
+                              int tiles_m, int tiles_n, int num_tiles, int nkb) {
   using Cfg = GemmCfg<BN>;
   int stage = 0;
   uint32_t phase = 0;
   for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-    const int m0 = (tile % tiles_m) * Cfg::BM;
-    const int n0 = (tile / tiles_m) * BN;
+    int mt, nt;
+    tile_coords(tile, tiles_m, tiles_n, mt, nt);
+    const int m0 = mt * Cfg::BM;
+    const int n0 = nt * BN;
     for (int kb = 0; kb < nkb; ++kb) {
       if (!mbar_wait(sm.empty(stage), phase ^ 1u, sm.abort_flag())) return;
+      VITQ_TRACE_EV(1);  // producer: stage free, issuing loads
       mbar_arrive_expect_tx(sm.full(stage), Cfg::STAGE_BYTES);
       tma_load_2d(sm.a(stage), tmA, kb * Cfg::BK, m0, sm.full(stage));
       tma_load_2d(sm.b(stage), tmB, kb * Cfg::BK, n0, sm.full(stage));
@@ -107,7 +129,9 @@ __device__ void gemm_mma(const GemmSmem<BN>& sm, uint32_t tmem_base, int num_til
       const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
       if (!mbar_wait(sm.tempty(buf), aph ^ 1u, sm.abort_flag())) return;
       tc_fence_after();
+      VITQ_TRACE_EV(2);  // mma: TMEM buffer free
       if (!mbar_wait(sm.full(stage), phase, sm.abort_flag())) return;
+      VITQ_TRACE_EV(3);  // mma: operands landed
       tc_fence_after();
       const uint32_t a0 = sm.a(stage), b0 = sm.b(stage);
 #pragma unroll
@@ -126,45 +150,81 @@ __device__ void gemm_mma(const GemmSmem<BN>& sm, uint32_t tmem_base, int num_til
   }
 }
 
+__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 unpack2(uint64_t v) {
+  float2 f;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+  return f;
+}
+// acc (two fp32 lanes) += p * s, one packed FMA.
+__device__ __forceinline__ uint64_t fma2(uint64_t p, uint64_t s, uint64_t acc) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(p), "l"(s), "l"(acc));
+  return d;
+}
+
 template <int BN>
 __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const GemmArgs& g,
-                              int tiles_m, int num_tiles, int nkb) {
+                              int tiles_m, int tiles_n, int num_tiles, int nkb) {
   using Cfg = GemmCfg<BN>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int quad = warp & 3;               // TMEM lane quadrant this warp may access
-  const int cg = (warp - 2) >> 2;          // which 128-column half of the tile
+  const int quad = warp & 3;                         // TMEM lane quadrant this warp may access
+  const int cg = (warp - Cfg::EPI_WARP0) >> 2;       // which 128-column group of the tile
   const int r_in = quad * 32 + lane;
   uint32_t cnt = 0;
   for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-    const int m0 = (tile % tiles_m) * Cfg::BM;
-    const int n0 = (tile / tiles_m) * BN;
+    int mt, nt;
+    tile_coords(tile, tiles_m, tiles_n, mt, nt);
+    const int m0 = mt * Cfg::BM;
+    const int n0 = nt * BN;
     const int row = m0 + r_in;
     const int col0 = n0 + cg * 128;
     const bool row_ok = row < g.M;
     const bool col_ok = col0 < g.N;
-    float acc[128];
+    const float* sa_ptr = g.sA + row;
+    const float* sw_ptr = g.sW + (size_t)(col0 >> 7) * nkb;
+    uint64_t acc[64];
 #pragma unroll
-    for (int j = 0; j < 128; ++j) acc[j] = 0.f;
+    for (int j = 0; j < 64; ++j) acc[j] = 0ull;
+    // scales are loaded one K block ahead so their latency hides behind the previous block
+    float sa_next = row_ok ? __ldg(sa_ptr) : 0.f;
+    float sw_next = col_ok ? __ldg(sw_ptr) : 0.f;
     for (int kb = 0; kb < nkb; ++kb, ++cnt) {
       const uint32_t buf = cnt % Cfg::NBUF;
       const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
-      const float sa = row_ok ? __ldg(g.sA + (size_t)kb * g.ldsA + row) : 0.f;
-      const float sw = col_ok ? __ldg(g.sW + (size_t)(col0 >> 7) * nkb + kb) : 0.f;
-      const float scale = sa * sw;
+      const float scale = sa_next * sw_next;
+      if (kb + 1 < nkb) {
+        sa_next = row_ok ? __ldg(sa_ptr + (size_t)(kb + 1) * g.ldsA) : 0.f;
+        sw_next = col_ok ? __ldg(sw_ptr + kb + 1) : 0.f;
+      }
+      const uint64_t s2 = pack2(scale, scale);
+      if (lane == 0) VITQ_TRACE_EV(4);  // epilogue: waiting for partial
       const bool ok = mbar_wait(sm.tfull(buf), aph, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
+      if (lane == 0) VITQ_TRACE_EV(5);  // epilogue: partial ready
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + cg * 128;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld32(taddr + c * 32, r);
+      for (int h = 0; h < 2; ++h) {
+        uint32_t r0[32], r1[32];
+        tmem_ld32(taddr + h * 64, r0);
+        tmem_ld32(taddr + h * 64 + 32, r1);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) acc[c * 32 + j] = fmaf(__uint_as_float(r[j]), scale, acc[c * 32 + j]);
+        for (int j = 0; j < 16; ++j) {
+          acc[h * 32 + j] = fma2(pack2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1])), s2,
+                                 acc[h * 32 + j]);
+          acc[h * 32 + 16 + j] = fma2(pack2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1])), s2,
+                                      acc[h * 32 + 16 + j]);
+        }
       }
       tc_fence_before();
       __syncwarp();
+      if (lane == 0) VITQ_TRACE_EV(6);  // epilogue: partial consumed
       if (lane == 0) mbar_arrive(sm.tempty(buf));
     }
     if (row_ok && col_ok) {
@@ -176,7 +236,11 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
         if (col < g.N) {
           float v[8];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) v[i] = acc[c8 * 8 + i];
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = unpack2(acc[c8 * 4 + i]);
+            v[2 * i] = f.x;
+            v[2 * i + 1] = f.y;
+          }
           if (g.bias) {
             const uint4 bu = __ldg(reinterpret_cast<const uint4*>(g.bias + col));
             const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
@@ -244,16 +308,18 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *sm.tmem_holder();
 
-  if (warp == 0) {
-    if (lane == 0) {
+  if (warp < Cfg::EPI_WARP0) {
+    if (Cfg::SPLIT_REGS) asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+    if (warp == 0 && lane == 0) {
       prefetch_tensormap(&tmA);
       prefetch_tensormap(&tmB);
-      gemm_producer<BN>(sm, &tmA, &tmB, tiles_m, num_tiles, nkb);
+      gemm_producer<BN>(sm, &tmA, &tmB, tiles_m, tiles_n, num_tiles, nkb);
+    } else if (warp == 1 && lane == 0) {
+      gemm_mma<BN>(sm, tmem_base, num_tiles, nkb);
     }
-  } else if (warp == 1) {
-    if (lane == 0) gemm_mma<BN>(sm, tmem_base, num_tiles, nkb);
   } else {
-    gemm_epilogue<BN>(sm, tmem_base, args, tiles_m, num_tiles, nkb);
+    if (Cfg::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
+    gemm_epilogue<BN>(sm, tmem_base, args, tiles_m, tiles_n, num_tiles, nkb);
   }
 
   tc_fence_before();
@@ -270,12 +336,15 @@ template <int BN>
 cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
                       cudaStream_t st) {
   using Cfg = GemmCfg<BN>;
-  static bool attr_done = false;  // per process; the attribute is per device function
-  if (!attr_done) {
-    cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)Cfg::SMEM);
+  cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)Cfg::SMEM);
+  if (e != cudaSuccess) return e;
+  if (Cfg::SPLIT_REGS) {
+    // setmaxnreg.inc only draws on the registers the CTA was launched with.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, fp8_gemm_kernel<BN>);
     if (e != cudaSuccess) return e;
-    attr_done = true;
+    if (fa.numRegs < Cfg::MIN_LAUNCH_REGS) return cudaErrorInvalidConfiguration;
   }
   const int tiles = ((a.M + 127) / 128) * ((a.N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;

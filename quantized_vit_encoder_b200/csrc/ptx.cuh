@@ -17,6 +17,29 @@ constexpr unsigned int kErrWaitTimeout = 1u;
 // A wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+// Event tracing for development builds (-DVITQ_TRACE): records (clock64, tag,
+// warp) for CTA 0 into a device buffer read by vitq_trace_read.  Compiles to
+// nothing in normal builds.
+#ifdef VITQ_TRACE
+constexpr unsigned kTraceCap = 1u << 16;
+__device__ unsigned long long g_trace[kTraceCap][2];
+__device__ unsigned int g_trace_n = 0;
+#define VITQ_TRACE_EV(tag)                                                        \
+  do {                                                                            \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {                  \
+      unsigned i_ = atomicAdd(&g_trace_n, 1u);                                    \
+      if (i_ < kTraceCap) {                                                       \
+        g_trace[i_][0] = clock64();                                               \
+        g_trace[i_][1] = ((unsigned long long)(tag) << 16) | (threadIdx.x >> 5);  \
+      }                                                                           \
+    }                                                                             \
+  } while (0)
+#else
+#define VITQ_TRACE_EV(tag) \
+  do {                     \
+  } while (0)
+#endif
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -30,12 +30,24 @@ def rel_l2(a, b):
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
 
 
+def bf16_ulp(v):
+    """Spacing of bf16 values at |v| (2^(e-7) for |v| in [2^e, 2^(e+1)))."""
+    v = np.abs(np.asarray(v, np.float64))
+    e = np.floor(np.log2(np.maximum(v, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
 def assert_close(got, want, rel=REL_L2, mabs=MAX_ABS, what=""):
+    """rel-L2 <= rel, and every element within max(mabs, one bf16 ulp of the reference):
+    a bf16 output cannot be closer than one rounding step, which exceeds 3e-2 for |v| >= 4."""
     got, want = np.asarray(got, np.float64), np.asarray(want, np.float64)
     assert got.shape == want.shape, (what, got.shape, want.shape)
     assert np.all(np.isfinite(got)), what
-    r, m = rel_l2(got, want), float(np.max(np.abs(got - want))) if got.size else 0.0
-    assert r <= rel and m <= mabs, f"{what}: rel_l2={r:.3e} max_abs={m:.3e}"
+    r = rel_l2(got, want)
+    d = np.abs(got - want)
+    m = float(d.max()) if got.size else 0.0
+    worst = float((d / np.maximum(mabs, bf16_ulp(want))).max()) if got.size else 0.0
+    assert r <= rel and worst <= 1.0, f"{what}: rel_l2={r:.3e} max_abs={m:.3e} (worst/allowed {worst:.2f})"
     return r, m
 
 
@@ -115,6 +127,31 @@ def test_gelu_quant_bit_exact(lib, M, K):
     q, s = vitq.gelu_quant(f.cuda())
     qr, sr = ov.gelu_quant(f64(f))
     assert_codes_equal(q, s, qr, sr, f"gelu_quant {M}x{K}")
+
+
+def test_gelu_quant_wide_range_bands(lib):
+    """Rows of narrow x bands covering [-12, 9]: every group's scale follows its band, so the
+    codes see the bf16 GELU values everywhere, including the far negative tail."""
+    from quantized_vit_encoder_b200 import vitq
+    rows = 420
+    lo = torch.linspace(-12.0, 9.0, rows + 1)[:-1]
+    g = torch.Generator().manual_seed(45)
+    f = (lo[:, None] + torch.rand((rows, 256), generator=g) * 0.05).to(torch.bfloat16)
+    q, s = vitq.gelu_quant(f.cuda())
+    qr, sr = ov.gelu_quant(f64(f))
+    assert_codes_equal(q, s, qr, sr, "gelu wide")
+
+
+def test_ln_quant_offset_mean(lib):
+    """Rows with |mean| several times their spread (the one-pass variance is still exact enough)."""
+    from quantized_vit_encoder_b200 import vitq
+    M, K = 257, 1152
+    x = (wl.random_bf16((M, K), 46, 1.0).float() + torch.linspace(-8, 8, M)[:, None]).to(torch.bfloat16)
+    g = (1 + wl.random_bf16((K,), 47, 0.02).float()).to(torch.bfloat16)
+    b = wl.random_bf16((K,), 48, 0.01)
+    q, s = vitq.ln_quant(x.cuda(), g.cuda(), b.cuda())
+    qr, sr = ov.ln_quant(f64(x), f64(g), f64(b), 1e-6)
+    assert_codes_equal(q, s, qr, sr, "ln offset")
 
 
 # ----------------------------------------------------------------- GEMM

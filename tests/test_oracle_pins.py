@@ -257,6 +257,13 @@ def test_gelu_identities():
     assert np.allclose(gl - ov.gelu_tanh_f64(-x), x, atol=1e-12)       # odd part is x/2 twice
     assert abs(ov.gelu_tanh_f64(1.0) - 0.5 * (1 + math.tanh(math.sqrt(2 / math.pi) * 1.044715))) < 1e-15
     assert np.allclose(ov.gelu_tanh_f64(np.array([30.0, -30.0])), [30.0, 0.0])
+    # equals the tanh form where that form is accurate, and stays accurate beyond it
+    xm = np.linspace(-4, 4, 801)
+    tanh_form = 0.5 * xm * (1 + np.tanh(math.sqrt(2 / math.pi) * (xm + 0.044715 * xm ** 3)))
+    assert np.allclose(ov.gelu_tanh_f64(xm), tanh_form, rtol=1e-10, atol=1e-300)   # tanh form loses digits as x -> -4
+    x8 = -8.0                                       # 1 + tanh(u) cancels completely here in fp64
+    u8 = math.sqrt(2 / math.pi) * (x8 + 0.044715 * x8 ** 3)
+    assert abs(ov.gelu_tanh_f64(x8) - x8 * math.exp(2 * u8) / (1 + math.exp(2 * u8))) <= 1e-15 * abs(ov.gelu_tanh_f64(x8))
     # tanh-GELU stays within 1e-3 of the exact erf GELU on [-8, 8]
     erf_gelu = 0.5 * x * (1 + np.array([math.erf(v / math.sqrt(2)) for v in x]))
     assert np.max(np.abs(gl - erf_gelu)) < 1e-3
