@@ -178,10 +178,11 @@ def build_tower(W, device):
     return vitq.DeviceTower(blocks, mergers)
 
 
-def kernel_table(records) -> dict:
+def kernel_table(records, by_shape: bool = False) -> dict:
     out = {}
     for name, ms, fl, by in records:
-        e = out.setdefault(name, {"launches": 0, "ms": 0.0, "flops": 0.0, "bytes": 0.0})
+        key = f"{name}@{fl / 1e9:.1f}GF/{by / 1e6:.1f}MB" if by_shape else name
+        e = out.setdefault(key, {"launches": 0, "ms": 0.0, "flops": 0.0, "bytes": 0.0})
         e["launches"] += 1
         e["ms"] += ms
         e["flops"] += fl
@@ -291,7 +292,9 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     for _ in range(2):
         step()
     torch.cuda.synchronize(dev)
-    table = kernel_table(vitq.profile_stop())
+    records = vitq.profile_stop()
+    table = kernel_table(records)
+    shapes = kernel_table(records, by_shape=True)
 
     # end to end through the public API: pinned host input -> device, taps -> pinned host
     taps_host = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in taps]
@@ -335,6 +338,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "roofline": roofline(table, peaks),
         "kernels": {k: {"launches": v["launches"] // 2, "ms_per_step": v["ms"] / 2,
                         "share": v["ms"] / sum(t["ms"] for t in table.values())} for k, v in table.items()},
+        "kernel_shapes": {k: {"launches": v["launches"] // 2, "us_per_launch": 1e3 * v["ms"] / v["launches"]}
+                          for k, v in sorted(shapes.items(), key=lambda kv: -kv[1]["ms"])},
         "gpu_launches": int(launches),
         "clocks": clk.summary(),
         "e2e": {"value": world * fl["tower"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",

@@ -28,8 +28,8 @@ constexpr float kE4M3Max = 448.0f;
 __device__ __forceinline__ float e4m3_quotient(float y, float s, float r) {
   float q = y * r;
   const uint32_t b = __float_as_uint(q) & 0x7FFFFFFFu;
-  const int mid = (int)(b & 0xFFFFFu) - 0x80000;
-  if (b < 0x3C800000u || (mid <= 16 && mid >= -16)) q = __fdiv_rn(y, s);
+  // mantissa tail within 16 of 0x80000  <=>  ((b - 0x7FFF0) mod 2^20) <= 32
+  if (b < 0x3C800000u || ((b - 0x7FFF0u) & 0xFFFFFu) <= 32u) q = __fdiv_rn(y, s);
   return q;
 }
 
@@ -78,17 +78,6 @@ __device__ __forceinline__ double bf16_bits_to_f64(uint32_t h) {
   uint64_t bits = (uint64_t)(h & 0x8000u) << 48;
   if (e) bits |= ((uint64_t)(e + 896u) << 52) | ((uint64_t)(h & 0x7Fu) << 45);
   return __longlong_as_double((long long)bits);
-}
-
-// Distance from y to the nearest bf16 rounding midpoint, and its bf16 rounding.
-// Returns false when y is too small for the fp32 test (|y| < 2^-100).
-__device__ __forceinline__ bool bf16_round_margin(float y, float* yr, float* dist) {
-  const uint32_t ey = __float_as_uint(y) & 0x7F800000u;
-  *yr = __bfloat162float(__float2bfloat16_rn(y));
-  if (ey < (27u << 23)) return false;
-  const float half = __uint_as_float(ey - (8u << 23));  // half a bf16 ulp in y's binade
-  *dist = half - fabsf(y - *yr);
-  return true;
 }
 
 // Lane layout shared by the row kernels: a warp covers 256 columns per step;
@@ -148,53 +137,82 @@ __global__ void ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
-  uint4 raw[ITERS];
-#pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
+  // Rows of up to 8 steps stay in registers; wider rows (the merger's 4608) are
+  // read again from L1/L2 in the second pass.
+  constexpr bool kKeep = ITERS <= 8;
+  constexpr int kHeld = kKeep ? ITERS : 1;
+  const __nv_bfloat16* xr = x + (size_t)row * ldx;
+  auto load_step = [&](int it) {
     const int col = lane_col(it, lane);
-    raw[it] = col < K ? *reinterpret_cast<const uint4*>(x + (size_t)row * ldx + col) : make_uint4(0, 0, 0, 0);
+    return col < K ? *reinterpret_cast<const uint4*>(xr + col) : make_uint4(0, 0, 0, 0);
+  };
+  uint4 raw[kHeld];
+  if (kKeep) {
+#pragma unroll
+    for (int it = 0; it < kHeld; ++it) raw[it] = load_step(it);
   }
-  double s1 = 0.0, s2 = 0.0;
+  // exact fp64 sums of the bf16 inputs (bf16 -> fp32 -> fp64 is exact); 4 chains each
+  double s1[4] = {0.0, 0.0, 0.0, 0.0}, s2[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll
   for (int it = 0; it < ITERS; ++it) {
-    const uint32_t w[4] = {raw[it].x, raw[it].y, raw[it].z, raw[it].w};
+    float v[8];
+    unpack8(kKeep ? raw[kKeep ? it : 0] : load_step(it), v);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const double a = bf16_bits_to_f64(w[i] & 0xFFFFu), b = bf16_bits_to_f64(w[i] >> 16);
-      s1 += a + b;
-      s2 = fma(a, a, fma(b, b, s2));
+    for (int i = 0; i < 8; ++i) {
+      const double d = (double)v[i];
+      s1[i & 3] += d;
+      s2[i & 3] = fma(d, d, s2[i & 3]);
     }
   }
+  double t1 = (s1[0] + s1[1]) + (s1[2] + s1[3]), t2 = (s2[0] + s2[1]) + (s2[2] + s2[3]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
-    s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-    s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    t1 += __shfl_xor_sync(0xffffffffu, t1, o);
+    t2 += __shfl_xor_sync(0xffffffffu, t2, o);
   }
-  const double mean = s1 / (double)K;
-  const double var = fmax(s2 / (double)K - mean * mean, 0.0);
+  const double mean = t1 / (double)K;
+  const double var = fmax(t2 / (double)K - mean * mean, 0.0);
   const double rstd = 1.0 / sqrt(var + eps);
   const float mh = (float)mean, ml = (float)(mean - (double)mh), r32 = (float)rstd;
 #pragma unroll
   for (int it = 0; it < ITERS; ++it) {
     const int col = lane_col(it, lane);
     const bool ok = col < K;
+    const uint4 rv = kKeep ? raw[kKeep ? it : 0] : load_step(it);
     float v[8];
-    unpack8(raw[it], v);
+    unpack8(rv, v);
     if (ok) {
       float g[8], b[8];
       load8_bf16(gamma + col, g);
       load8_bf16(beta + col, b);
+      bool slow = false;
+      float t[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const float t = ((v[i] - mh) - ml) * r32;
-        const float y = fmaf(t, g[i], b[i]);
-        float yr, dist;
-        const float err = (fabsf(t * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;  // 2^-20
-        if (!bf16_round_margin(y, &yr, &dist) || dist <= err) {
-          const double yd = ((double)v[i] - mean) * rstd * (double)g[i] + (double)b[i];
-          yr = __bfloat162float(__double2bfloat16(yd));
-        }
+        t[i] = ((v[i] - mh) - ml) * r32;
+        const float y = fmaf(t[i], g[i], b[i]);
+        // fp32 error of y is below (|t g| + |b|) 2^-20; distance of y to the nearest
+        // bf16 rounding midpoint = half a bf16 ulp (from y's exponent) - |y - bf16(y)|
+        const float yr = __bfloat162float(__float2bfloat16_rn(y));
+        const float half = __uint_as_float((__float_as_uint(y) & 0x7F800000u) - (8u << 23));
+        const float err = (fabsf(t[i] * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;
+        slow |= (half - fabsf(y - yr) <= err) | (fabsf(y) < 1e-30f);
         v[i] = yr;
+      }
+      if (slow) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float y = fmaf(t[i], g[i], b[i]);
+          const float yr = __bfloat162float(__float2bfloat16_rn(y));
+          const float half = __uint_as_float((__float_as_uint(y) & 0x7F800000u) - (8u << 23));
+          const float err = (fabsf(t[i] * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;
+          if (half - fabsf(y - yr) <= err || fabsf(y) < 1e-30f) {
+            float xi[8];
+            unpack8(rv, xi);
+            const double yd = ((double)xi[i] - mean) * rstd * (double)g[i] + (double)b[i];
+            v[i] = __bfloat162float(__double2bfloat16(yd));
+          }
+        }
       }
     }
     quant_store(v, ok, lane, row, col, K, q, s, lds);
@@ -206,23 +224,34 @@ __global__ void ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
 // The fp32 sigmoid form (hardware exp2 and reciprocal) has no cancellation; its
 // relative error is below 2^-21 (|u| + 2) (measured against fp64 over x in
 // [-12, 9]).  When the result lies within 2^-20 (|u| + 4) |g| of a bf16 rounding
-// midpoint (or is too small for that test) it is recomputed in fp64, so the
-// bf16 result is the rounding of the fp64 value x / (1 + exp(-2u)).
+// midpoint (or is below 1e-30) it is recomputed in fp64, so the bf16 result is
+// the rounding of the fp64 value x / (1 + exp(-2u)).
 
-__device__ __forceinline__ float gelu_tanh_bf16(float x) {
-  const float u = x * fmaf(0.035677408136300125f, x * x, 0.7978845608028654f);
-  float e, rc;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-2.8853900817779268f * u));   // exp(-2u)
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.0f + e));
-  const float g = x * rc;
-  float gr, dist;
-  const float err = fabsf(g) * (fabsf(u) + 4.0f) * 9.5367431640625e-07f;  // 2^-20
-  if (!bf16_round_margin(g, &gr, &dist) || dist <= err) {
-    const double xd = (double)x;
-    const double ud = 0.79788456080286535588 * (xd + 0.044715 * xd * xd * xd);
-    gr = __bfloat162float(__double2bfloat16(xd / (1.0 + exp(-2.0 * ud))));
+__device__ __forceinline__ float gelu_f64_bf16(float x) {
+  const double xd = (double)x;
+  const double ud = 0.79788456080286535588 * (xd + 0.044715 * xd * xd * xd);
+  return __bfloat162float(__double2bfloat16(xd / (1.0 + exp(-2.0 * ud))));
+}
+
+// fp32 GELU of 8 values rounded to bf16; returns true if any of them lies within
+// its error bound of a bf16 rounding midpoint (then gelu_f64_bf16 decides it).
+__device__ __forceinline__ bool gelu8_fast(const float (&x)[8], float (&g)[8], bool (&slow)[8]) {
+  bool any = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float u = x[i] * fmaf(0.035677408136300125f, x[i] * x[i], 0.7978845608028654f);
+    float e, rc;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-2.8853900817779268f * u));   // exp(-2u)
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.0f + e));
+    const float gv = x[i] * rc;
+    const float gr = __bfloat162float(__float2bfloat16_rn(gv));
+    const float half = __uint_as_float((__float_as_uint(gv) & 0x7F800000u) - (8u << 23));
+    const float err = fabsf(gv) * (fabsf(u) + 4.0f) * 9.5367431640625e-07f;  // 2^-20 (|u| + 4) |g|
+    slow[i] = (half - fabsf(gv - gr) <= err) | (fabsf(gv) < 1e-30f);
+    any |= slow[i];
+    g[i] = gr;
   }
-  return gr;
+  return any;
 }
 
 __global__ void gelu_quant_kernel(const __nv_bfloat16* __restrict__ f, int M, int K, int ldf,
@@ -237,9 +266,14 @@ __global__ void gelu_quant_kernel(const __nv_bfloat16* __restrict__ f, int M, in
   const bool ok = col < K;
   float v[8];
   if (ok) {
-    load8_bf16(f + (size_t)row * ldf + col, v);
+    float xv[8];
+    bool slow[8];
+    load8_bf16(f + (size_t)row * ldf + col, xv);
+    if (gelu8_fast(xv, v, slow)) {
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = gelu_tanh_bf16(v[i]);
+      for (int i = 0; i < 8; ++i)
+        if (slow[i]) v[i] = gelu_f64_bf16(xv[i]);
+    }
   } else {
 #pragma unroll
     for (int i = 0; i < 8; ++i) v[i] = 0.f;

@@ -2,7 +2,8 @@
 
     python -m quantized_vit_encoder_b200.profile_case STAGE [--iters N]
 
-STAGE: attention | gemm_qkv | gemm_proj | gemm_fc1 | gemm_fc2 | ln_quant | gelu_quant | rope | block.
+STAGE: attention | gemm_qkv | gemm_proj | gemm_fc1 | gemm_fc2 | ln_quant | ln_quant_merger |
+       quant_act | gelu_quant | rope | block.
 Device memory stays below 0.5 GB; each iteration is one launch of the stage's
 kernel (block: the ten launches of one block).
 """
@@ -50,6 +51,13 @@ def main():
         run = lambda: vitq.fp8_block_gemm(qa, sa, t[name + "_q"], t[name + "_s"], t[name + "_b"], res, out)  # noqa: E731
     elif a.stage == "ln_quant":
         run = lambda: vitq.ln_quant(x, t["norm1_w"], t["norm1_b"])  # noqa: E731
+    elif a.stage == "ln_quant_merger":
+        xm = x.view(n // 4, 4608)
+        g = (1 + wl.random_bf16((4608,), 6, 0.02).float()).to(torch.bfloat16).to(dev)
+        b = wl.random_bf16((4608,), 7, 0.01).to(dev)
+        run = lambda: vitq.ln_quant(xm, g, b)  # noqa: E731
+    elif a.stage == "quant_act":
+        run = lambda: vitq.quant_act(x)  # noqa: E731
     elif a.stage == "gelu_quant":
         f = wl.random_bf16((n, 4304), 4, 1.0).to(dev)
         run = lambda: vitq.gelu_quant(f)  # noqa: E731
