@@ -170,6 +170,28 @@ int vit_merger_forward(const vitq_merger_weights* w, const void* x, int n_tokens
                        size_t ws_bytes, void* stream);
 size_t vitq_merger_workspace_bytes(int n_tokens);
 
+/* The merger above with no workspace argument and no allocation of any kind.
+ * This entry point has no counterpart in the sources: it serves callers that
+ * may not allocate device memory, or pass a buffer, once running (code inside
+ * an allocator callback, a plugin host that forbids allocations after
+ * start-up, a serving loop that must never reach cudaMalloc, which can
+ * synchronise the whole device).  Its scratch is one fixed array per device,
+ * part of this library, sized for VITQ_MERGER_STATIC_MAX_TOKENS input tokens
+ * (about 13.6 MiB).
+ *  - n_tokens > VITQ_MERGER_STATIC_MAX_TOKENS returns VITQ_ERR_WORKSPACE and
+ *    launches nothing; other arguments as vit_merger_forward.
+ *  - The first call on each device, with that device current, looks up the
+ *    array's device address (and may load this library's kernels there).
+ *    Make that first call before any stream capture begins.
+ *  - All calls on one device share the array.  Calls issued in order on one
+ *    stream are safe; calls that can overlap (different streams, or host
+ *    threads, without ordering between them) race on it and corrupt each
+ *    other's results.
+ *  - Nothing in the array needs to start at zero. */
+#define VITQ_MERGER_STATIC_MAX_TOKENS 4096
+int vit_merger_forward_static(const vitq_merger_weights* w, const void* x, int n_tokens, void* out,
+                              void* stream);
+
 /* The 27-block tower over packed images with DeepStack taps ([FRT] s3 "DeepStack
  * taps at layers 8 / 16 / 24", [VE] deepstack_indexes [8,16,24] + final merger).
  * x: bf16 [n, 1152] patch embeddings, overwritten with the block-27 output.

@@ -3,3 +3,4 @@
 #include "gemm_fp8.cu"
 #include "attention.cu"
 #include "api.cu"
+#include "merger_static.cu"

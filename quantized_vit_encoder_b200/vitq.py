@@ -52,6 +52,7 @@ _SIGS = {
     "vit_block_forward": [C.POINTER(BlockWeights), _vp, _i, _vp, _i, _i, _vp, _vp, _sz, _vp],
     "vitq_block_workspace_bytes": [_i],
     "vit_merger_forward": [C.POINTER(MergerWeights), _vp, _i, _vp, _vp, _sz, _vp],
+    "vit_merger_forward_static": [C.POINTER(MergerWeights), _vp, _i, _vp, _vp],
     "vitq_merger_workspace_bytes": [_i],
     "vit_tower_forward": [C.POINTER(TowerWeights), _vp, _vp, _i, C.POINTER(_vp), _vp, _sz, _vp],
     "vitq_tower_workspace_bytes": [_i, _i],
@@ -278,6 +279,17 @@ def merger_forward(mg: DeviceMerger, x, ws, out=None, stream=None):
         out = torch.empty((n // 4, OUT_HIDDEN), dtype=torch.bfloat16, device=x.device)
     _check(load().vit_merger_forward(C.byref(mg.struct), _p(x), n, _p(out), _p(ws), ws.numel(), _stream(stream)),
            "vit_merger_forward")
+    return out
+
+
+MERGER_STATIC_MAX_TOKENS = 4096
+
+
+def merger_forward_static(mg: DeviceMerger, x, out):
+    """vit_merger_forward_static: the merger with the library's fixed scratch
+    (no workspace, no allocation); out must be given, bf16 [n/4, 2048]."""
+    _check(load().vit_merger_forward_static(C.byref(mg.struct), _p(x), x.shape[0], _p(out), _stream(None)),
+           "vit_merger_forward_static")
     return out
 
 
