@@ -545,17 +545,15 @@ const char* vitq_status_string(int s) {
 unsigned long long vitq_launch_count(void) { return g_launches.load(); }
 
 #ifdef VITQ_TRACE
-// Development builds only: copies up to cap (clock, tag<<16|warp) records and clears the buffer.
+// Development builds only: copies the [32][4096] clock table (0 = no event) and clears it.
 int vitq_trace_read(unsigned long long* out, int cap) {
   cudaDeviceSynchronize();
-  unsigned int n = 0;
-  cudaMemcpyFromSymbol(&n, g_trace_n, sizeof(n));
-  if (n > kTraceCap) n = kTraceCap;
-  if ((int)n > cap) n = (unsigned)cap;
-  cudaMemcpyFromSymbol(out, g_trace, (size_t)n * 16);
-  const unsigned int zero = 0;
-  cudaMemcpyToSymbol(g_trace_n, &zero, sizeof(zero));
-  return (int)n;
+  const int n = (int)(kTraceTags * kTracePerTag);
+  if (cap < n) return -1;
+  cudaMemcpyFromSymbol(out, g_trace, (size_t)n * 8);
+  static std::vector<unsigned long long> zero((size_t)n, 0ull);
+  cudaMemcpyToSymbol(g_trace, zero.data(), (size_t)n * 8);
+  return n;
 }
 #endif
 

@@ -12,13 +12,20 @@
 //     softmax of S_x(j) runs (the softmax frees S_x once it holds it in
 //     registers), and the two tiles interleave on the tensor core;
 //   * the softmax exponentials run on MUFU ex2; a share can move to a polynomial
-//     on the FMA pipe (kPolyEvery) to balance the two pipes;
-//   * Q, K, V are read straight from the packed qkv activation [n, 3, 16, 72]
+//     on the FMA pipe (kPolyEvery) to balance the two pipes.  The two softmax
+//     warps that share an SMSP (tile A and tile B) take turns for their
+//     exponentials, so each turn has MUFU to itself while the other warp reads
+//     its next scores and waits for its P.V;
+//   * K and V are read straight from the packed qkv activation [n, 3, 16, 72]
 //     through 3D TMA maps (d, slot, token).  head_dim 72 is padded to 80 by
-//     the tensor map itself: d 0..63 land in a 128B-swizzled tile and d 64..79
-//     in a 32B-swizzled tile, and d >= 72 lies outside the map so TMA fills
-//     zeros.  The padding never exists in HBM;
-//   * S = Q K^T runs as 5 tcgen05.mma (K = 16 each) into the tile's TMEM S buffer;
+//     the tensor map itself: d >= 72 lies outside the map so TMA fills zeros,
+//     and the padding never exists in HBM.  K: d 0..63 in a 128B-swizzled tile,
+//     d 64..79 in a 32B-swizzled tile.  V: d 0..63 and d 64..127 in two
+//     128B-swizzled tiles, so that P.V is one N = 80 MMA per 16 keys (two
+//     MMAs of N = 64 and 16 cost twice as much: each re-reads P);
+//   * each softmax thread copies its Q row into TMEM once (columns packed two
+//     bf16 per 32-bit column), and S = Q K^T runs as 5 tcgen05.mma with A in
+//     TMEM (K = 16 each) into the tile's TMEM S buffer;
 //   * the softmax warps keep a running max in the log2 domain and rescale O
 //     (in TMEM) only when the max grows by more than 8, write P as bf16 into a
 //     128B-swizzled shared tile, and the MMA warp accumulates O += P V with V
@@ -33,21 +40,23 @@ namespace vitq {
 namespace {
 
 constexpr int kBM = 128, kBN = 128, kStages = 3, kQTiles = 2;
-// Shared memory: Q tiles (A, B), a ring of K/V stages, the P tiles (A, B).
-constexpr int kQBytes = 20480;                          // 128 x 64 (SW128) + 128 x 16 (SW32), bf16
-constexpr int kQLo = 0, kQHi = 16384;                   // offsets inside a Q tile
-constexpr int kKV0 = kQTiles * kQBytes, kKVStride = 40960;
-constexpr int kKLo = 0, kKHi = 16384, kVLo = 20480, kVHi = 36864;
+// Shared memory: a ring of K/V stages, the P tiles (A, B).
+constexpr int kKV0 = 0, kKVStride = 53248;
+constexpr int kKLo = 0, kKHi = 16384, kVLo = 20480, kVHi = 36864;   // V hi = V lo + 16384 (N-atom stride)
 constexpr int kP0 = kKV0 + kStages * kKVStride;         // P tile X: two 64-key atoms of 16 KB
 constexpr int kPBytes = 32768;
 constexpr int kBar = kP0 + kQTiles * kPBytes;
-// barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], s_free[2]
-constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles;
+// barriers: slot 0 (unused), kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2],
+// s_free[2], turn[2][4] (softmax warp of tile x on SMSP q finished its
+// exponentials), q_ready[2] (Q tile x is in TMEM)
+constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles;
 constexpr size_t kAttnSmem = 1024 + kBar + kNumBars * 8 + 16;
 static_assert(kAttnSmem <= 232448, "shared memory budget");
-// TMEM columns: S_A 0..127, S_B 128..255, O_A 256..335, O_B 384..463.
+// TMEM columns: S_A 0..127, S_B 128..255, O_A 256..335, Q_A 336..383, O_B 384..463,
+// Q_B 464..511 (Q: 40 columns of bf16 pairs, written as 48).
 __device__ __forceinline__ uint32_t tmem_s(int x) { return (uint32_t)x * 128u; }
 __device__ __forceinline__ uint32_t tmem_o(int x) { return 256u + (uint32_t)x * 128u; }
+__device__ __forceinline__ uint32_t tmem_q(int x) { return 336u + (uint32_t)x * 128u; }
 // Warpgroup 0: warp 0 TMA producer, warps 1 and 2 MMA issuers for Q tiles A
 // and B (warp 3 idle); warpgroups 1 and 2: softmax of Q tiles A and B.
 constexpr int kThreads = 128 * (1 + kQTiles);
@@ -60,6 +69,7 @@ constexpr int kPolyEvery = VITQ_ATTN_POLY_EVERY;
 constexpr int kPolyMod = kPolyEvery > 0 ? kPolyEvery : 1;
 
 struct AttnArgs {
+  const __nv_bfloat16* qkv;
   const int32_t* cu;
   __nv_bfloat16* out;
   int n_tokens;
@@ -82,18 +92,18 @@ struct AttnSmem {
   uint8_t* base;
   __device__ uint32_t at(int off) const { return smem_u32(base + off); }
   __device__ uint64_t* bar(int i) const { return reinterpret_cast<uint64_t*>(base + kBar) + i; }
-  __device__ uint32_t q_full() const { return smem_u32(bar(0)); }
+  __device__ uint32_t q_ready(int x) const { return smem_u32(bar(1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + x)); }
   __device__ uint32_t kv_full(int s) const { return smem_u32(bar(1 + s)); }
   __device__ uint32_t kv_empty(int s) const { return smem_u32(bar(1 + kStages + s)); }
   __device__ uint32_t s_full(int x) const { return smem_u32(bar(1 + 2 * kStages + x)); }
   __device__ uint32_t p_full(int x) const { return smem_u32(bar(1 + 2 * kStages + kQTiles + x)); }
   __device__ uint32_t pv_done(int x) const { return smem_u32(bar(1 + 2 * kStages + 2 * kQTiles + x)); }
   __device__ uint32_t s_free(int x) const { return smem_u32(bar(1 + 2 * kStages + 3 * kQTiles + x)); }
+  __device__ uint32_t turn(int x, int q) const { return smem_u32(bar(1 + 2 * kStages + 4 * kQTiles + x * 4 + q)); }
   __device__ uint32_t* tmem_holder() const { return reinterpret_cast<uint32_t*>(bar(kNumBars)); }
   __device__ volatile int* abort_flag() const {
     return reinterpret_cast<volatile int*>(tmem_holder() + 1);
   }
-  __device__ uint32_t q(int x, int part) const { return at(x * kQBytes + part); }
   __device__ uint32_t kv(int s, int part) const { return at(kKV0 + s * kKVStride + part); }
   __device__ uint32_t p(int x) const { return at(kP0 + x * kPBytes); }
 };
@@ -151,59 +161,52 @@ __device__ __forceinline__ float2 ex2_poly2(float x0, float x1) {
 
 
 __device__ void attn_producer(const AttnSmem& sm, const CUtensorMap* tlo, const CUtensorMap* thi,
-                              int head, int q_row, int n_q, int kv_row0, int n_kv, int off) {
-  mbar_arrive_expect_tx(sm.q_full(), kQBytes * n_q);
-  for (int x = 0; x < n_q; ++x) {
-    tma_load_3d(sm.q(x, kQLo), tlo, 0, head, q_row + x * kBM, sm.q_full());
-    tma_load_3d(sm.q(x, kQHi), thi, 64, head, q_row + x * kBM, sm.q_full());
-  }
+                              int head, int kv_row0, int n_kv, int off) {
   for (int j = 0; j < n_kv; ++j) {
     const int s = j % kStages;
     const uint32_t ph = (uint32_t)(j / kStages) & 1u;
     if (!mbar_wait(sm.kv_empty(s), ph ^ 1u, sm.abort_flag())) return;
-    mbar_arrive_expect_tx(sm.kv_full(s), 40960);
+    mbar_arrive_expect_tx(sm.kv_full(s), kKVStride);
     const int row = kv_row0 + kv_tile(j, off, n_kv) * kBN;
     tma_load_3d(sm.kv(s, kKLo), tlo, 0, 16 + head, row, sm.kv_full(s));
     tma_load_3d(sm.kv(s, kKHi), thi, 64, 16 + head, row, sm.kv_full(s));
     tma_load_3d(sm.kv(s, kVLo), tlo, 0, 32 + head, row, sm.kv_full(s));
-    tma_load_3d(sm.kv(s, kVHi), thi, 64, 32 + head, row, sm.kv_full(s));
+    tma_load_3d(sm.kv(s, kVHi), tlo, 64, 32 + head, row, sm.kv_full(s));   // d 64..127, >= 72 zero
   }
 }
 
-// S_x = Q_x K_j^T (5 MMAs of K = 16 over the padded head_dim 80) into S buffer x.
+// S_x = Q_x K_j^T (5 MMAs of K = 16 over the padded head_dim 80, Q from TMEM) into S buffer x.
 __device__ bool attn_issue_s(const AttnSmem& sm, uint32_t tmem, int x, int j) {
   constexpr uint32_t idesc = make_idesc(1, 1, 0, 0, 128, 128);
   const int s = j % kStages;
   if (!mbar_wait(sm.kv_full(s), (uint32_t)(j / kStages) & 1u, sm.abort_flag())) return false;
   tc_fence_after();
-  const uint32_t d = tmem + tmem_s(x);
-  const uint32_t qlo = sm.q(x, kQLo), klo = sm.kv(s, kKLo);
+  const uint32_t d = tmem + tmem_s(x), q = tmem + tmem_q(x);
+  const uint32_t klo = sm.kv(s, kKLo);
 #pragma unroll
   for (int k = 0; k < 4; ++k)
-    mma_bf16_ss(d, make_smem_desc(qlo + 32 * k, 16, 1024, kSwizzle128B),
-                make_smem_desc(klo + 32 * k, 16, 1024, kSwizzle128B), idesc, k > 0 ? 1u : 0u);
-  mma_bf16_ss(d, make_smem_desc(sm.q(x, kQHi), 16, 256, kSwizzle32B),
-              make_smem_desc(sm.kv(s, kKHi), 16, 256, kSwizzle32B), idesc, 1u);
+    mma_bf16_ts(d, q + 8 * k, make_smem_desc(klo + 32 * k, 16, 1024, kSwizzle128B), idesc, k > 0 ? 1u : 0u);
+  mma_bf16_ts(d, q + 32, make_smem_desc(sm.kv(s, kKHi), 16, 256, kSwizzle32B), idesc, 1u);
   tc_commit(sm.s_full(x));
   return true;
 }
 
-// O_x += P_x V_j: P from shared memory (K-major), V MN-major; N = 64 + 16.
+// O_x += P_x V_j: P from shared memory (K-major), V MN-major in two 64-wide
+// atoms (LBO 16384 bytes apart); one N = 80 MMA per 16 keys.
 template <bool kVF16>
 __device__ bool attn_issue_pv(const AttnSmem& sm, uint32_t tmem, int x, int j) {
   constexpr uint32_t fmt = kVF16 ? 0u : 1u;
-  constexpr uint32_t idesc_lo = make_idesc(fmt, fmt, 0, 1, 128, 64);
-  constexpr uint32_t idesc_hi = make_idesc(fmt, fmt, 0, 1, 128, 16);
+  constexpr uint32_t idesc = make_idesc(fmt, fmt, 0, 1, 128, 80);
   if (!mbar_wait(sm.p_full(x), (uint32_t)j & 1u, sm.abort_flag())) return false;
+  VITQ_TRACE_EV(14 + x, j);   // mma: P complete
   tc_fence_after();
   const int s = j % kStages;
-  const uint32_t vlo = sm.kv(s, kVLo), vhi = sm.kv(s, kVHi), p0 = sm.p(x);
+  const uint32_t vlo = sm.kv(s, kVLo), p0 = sm.p(x);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const uint64_t ad = make_smem_desc(p0 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B);
     const uint32_t acc = (j > 0 || k > 0) ? 1u : 0u;
-    mma_bf16_ss(tmem + tmem_o(x), ad, make_smem_desc(vlo + k * 2048, 16384, 1024, kSwizzle128B), idesc_lo, acc);
-    mma_bf16_ss(tmem + tmem_o(x) + 64, ad, make_smem_desc(vhi + k * 512, 4096, 256, kSwizzle32B), idesc_hi, acc);
+    mma_bf16_ss(tmem + tmem_o(x), ad, make_smem_desc(vlo + k * 2048, kVHi - kVLo, 1024, kSwizzle128B), idesc, acc);
   }
   tc_commit(sm.pv_done(x));
   return true;
@@ -216,17 +219,19 @@ __device__ bool attn_issue_pv(const AttnSmem& sm, uint32_t tmem, int x, int j) {
 // both tiles' P.V of that stage have completed (kv_empty counts one commit per tile).
 template <bool kVF16>
 __device__ void attn_mma(const AttnSmem& sm, uint32_t tmem, int x, int n_kv) {
-  if (!mbar_wait(sm.q_full(), 0, sm.abort_flag())) return;
+  if (!mbar_wait(sm.q_ready(x), 0, sm.abort_flag())) return;
+  tc_fence_after();
   if (!attn_issue_s(sm, tmem, x, 0)) return;
   for (int j = 0; j < n_kv; ++j) {
     if (j + 1 < n_kv) {
       if (!mbar_wait(sm.s_free(x), (uint32_t)j & 1u, sm.abort_flag())) return;
+      VITQ_TRACE_EV(16 + x, j);   // mma: S buffer free
       tc_fence_after();
       if (!attn_issue_s(sm, tmem, x, j + 1)) return;
-      VITQ_TRACE_EV(10 + x);   // mma: S issued
+      VITQ_TRACE_EV(10 + x, j + 1);   // mma: S issued
     }
     if (!attn_issue_pv<kVF16>(sm, tmem, x, j)) return;
-    VITQ_TRACE_EV(12 + x);     // mma: P.V issued
+    VITQ_TRACE_EV(12 + x, j);     // mma: P.V issued
     tc_commit(sm.kv_empty(j % kStages));
   }
 }
@@ -243,7 +248,7 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi, bool f16) {
 // TMEM twice (row max, then exponentials), 64 columns at a time, so a thread
 // holds at most 64 scores in registers.
 template <bool kVF16>
-__device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& g, int x, int head,
+__device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& g, int x, int n_q, int head,
                              int seq_start, int seq_len, int q0, int n_kv, int off) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;
@@ -251,11 +256,32 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
   const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
   const uint32_t s_addr = tmem + lane_addr + tmem_s(x), o_addr = tmem + lane_addr + tmem_o(x);
   uint8_t* pbase = sm.base + kP0 + x * kPBytes;
+  {
+    // this thread's Q row -> TMEM (bf16 pairs in columns 0..35, zeros up to 47)
+    uint32_t qw[3][16];
+    const bool q_ok = q0 + r < seq_len && seq_start + q0 + r < g.n_tokens;
+    const uint4* src = reinterpret_cast<const uint4*>(g.qkv + (size_t)(seq_start + q0 + r) * 3456 + head * 72);
+#pragma unroll
+    for (int i = 0; i < 12; ++i) {
+      const uint4 v = (q_ok && i < 9) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
+      qw[i >> 2][(i & 3) * 4 + 0] = v.x;
+      qw[i >> 2][(i & 3) * 4 + 1] = v.y;
+      qw[i >> 2][(i & 3) * 4 + 2] = v.z;
+      qw[i >> 2][(i & 3) * 4 + 3] = v.w;
+    }
+    const uint32_t q_addr = tmem + lane_addr + tmem_q(x);
+#pragma unroll
+    for (int c = 0; c < 3; ++c) tmem_st16(q_addr + c * 16, qw[c]);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.q_ready(x));
+  }
   float m_run = -INFINITY, l_run = 0.f;
   for (int j = 0; j < n_kv; ++j) {
     bool ok = mbar_wait(sm.s_full(x), (uint32_t)j & 1u, sm.abort_flag());
     if (!__all_sync(0xffffffffu, ok)) return;
-    if (lane == 0 && quad == 0) VITQ_TRACE_EV(20 + x);   // softmax: S ready
+    if (lane == 0 && quad == 0) VITQ_TRACE_EV(20 + x, j);   // softmax: S ready
     tc_fence_after();
     const int valid = seq_len - kv_tile(j, off, n_kv) * kBN;   // keys of this tile inside the segment
     // one TMEM round trip: all 128 scores of the row, then S_x is free for S_x(j+1)
@@ -263,6 +289,7 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
 #pragma unroll
     for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, su[c]);
     tmem_wait_ld();
+    if (lane == 0 && quad == 0) VITQ_TRACE_EV(26 + x, j);   // softmax: S in registers
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.s_free(x));
@@ -288,7 +315,7 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
       if (!__all_sync(0xffffffffu, ok)) return;
       tc_fence_after();
     }
-    if (lane == 0 && quad == 0) VITQ_TRACE_EV(22 + x);   // softmax: max known, O stable
+    if (lane == 0 && quad == 0) VITQ_TRACE_EV(22 + x, j);   // softmax: max known, O stable
     // new running max: it changes only when the tile max exceeds it by more than 8
     // (so P <= 2^8), and the decision is warp-uniform because the O rescale uses
     // warp-collective tcgen05.ld/st (rows that keep their max get alpha = 1).
@@ -304,6 +331,14 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
         m_run = mx;
       }
     }
+    // The two tiles' softmax warps on one SMSP take turns for the exponentials
+    // (A(j), B(j), A(j+1), ...): MUFU runs one tile at full rate while the other
+    // tile loads its scores, takes the row max and waits for its P.V.
+    if (n_q == 2 && (x == 1 || j > 0)) {
+      ok = mbar_wait(sm.turn(1 - x, quad), (uint32_t)(x == 1 ? j : j - 1) & 1u, sm.abort_flag());
+      if (!__all_sync(0xffffffffu, ok)) return;
+    }
+    if (lane == 0 && quad == 0) VITQ_TRACE_EV(28 + x, j);   // softmax: turn for the exponentials
     // P = 2^(s * scale_log2 - m_run), rounded to the P.V operand type, into the swizzled
     // P tile (64-key atom a holds keys 64a..64a+63); 8 fp32 partial row sums.
     const uint64_t sc2 = f2pack(g.scale_log2, g.scale_log2), nm2 = f2pack(-m_run, -m_run);
@@ -334,6 +369,10 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
         *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
+    if (n_q == 2 && !(x == 1 && j == n_kv - 1)) {   // hand the turn to the other tile
+      __syncwarp();
+      if (lane == 0) mbar_arrive(sm.turn(x, quad));
+    }
     if (rescale) {
       // O (complete up to P.V(j-1)) to the new max; done after P so the scores are dead
       uint32_t u[5][16];
@@ -355,7 +394,7 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0 && quad == 0) VITQ_TRACE_EV(24 + x);   // softmax: P written
+    if (lane == 0 && quad == 0) VITQ_TRACE_EV(24 + x, j);   // softmax: P written
     if (lane == 0) mbar_arrive(sm.p_full(x));
   }
   bool ok = mbar_wait(sm.pv_done(x), (uint32_t)(n_kv - 1) & 1u, sm.abort_flag());
@@ -400,12 +439,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    mbar_init(sm.q_full(), 1);
     for (int s = 0; s < kStages; ++s) {
       mbar_init(sm.kv_full(s), 1);
       mbar_init(sm.kv_empty(s), (uint32_t)n_q);       // one commit per active Q tile
     }
     for (int x = 0; x < kQTiles; ++x) {
+      for (int q = 0; q < 4; ++q) mbar_init(sm.turn(x, q), 1);
+      mbar_init(sm.q_ready(x), 4);
       mbar_init(sm.s_full(x), 1);
       mbar_init(sm.p_full(x), 4);
       mbar_init(sm.pv_done(x), 1);
@@ -426,13 +466,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
       prefetch_tensormap(&tlo);
       prefetch_tensormap(&thi);
-      attn_producer(sm, &tlo, &thi, head, seq_start + q0, n_q, seq_start, n_kv, off);
+      attn_producer(sm, &tlo, &thi, head, seq_start, n_kv, off);
     } else if ((warp == 1 || warp == 2) && lane == 0 && warp - 1 < n_q) {
       attn_mma<kVF16>(sm, tmem, warp - 1, n_kv);
     }
   } else {
     const int x = (warp >> 2) - 1;
-    if (x < n_q) attn_softmax<kVF16>(sm, tmem, args, x, head, seq_start, seq_len, q0 + x * kBM, n_kv, off);
+    if (x < n_q) attn_softmax<kVF16>(sm, tmem, args, x, n_q, head, seq_start, seq_len, q0 + x * kBM, n_kv, off);
   }
   tc_fence_before();
   __syncthreads();
@@ -457,7 +497,7 @@ cudaError_t launch_attention(const __nv_bfloat16* qkv, int n_tokens, const int32
   auto kern = v_f16 ? attn_kernel<true> : attn_kernel<false>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
   if (e != cudaSuccess) return e;
-  AttnArgs a{cu, out, n_tokens, scale * 1.4426950408889634f};
+  AttnArgs a{qkv, cu, out, n_tokens, scale * 1.4426950408889634f};
   dim3 grid((max_seqlen + kBM * kQTiles - 1) / (kBM * kQTiles), 16, n_seqs);
   kern<<<grid, kThreads, kAttnSmem, st>>>(tlo, thi, a);
   return cudaGetLastError();

@@ -104,7 +104,7 @@ __device__ void gemm_producer(const GemmSmem<BN>& sm, const CUtensorMap* tmA, co
     const int n0 = nt * BN;
     for (int kb = 0; kb < nkb; ++kb) {
       if (!mbar_wait(sm.empty(stage), phase ^ 1u, sm.abort_flag())) return;
-      VITQ_TRACE_EV(1);  // producer: stage free, issuing loads
+      VITQ_TRACE_EV(1, (tile - (int)blockIdx.x) / (int)gridDim.x * nkb + kb);  // producer: stage free, issuing loads
       mbar_arrive_expect_tx(sm.full(stage), Cfg::STAGE_BYTES);
       tma_load_2d(sm.a(stage), tmA, kb * Cfg::BK, m0, sm.full(stage));
       tma_load_2d(sm.b(stage), tmB, kb * Cfg::BK, n0, sm.full(stage));
@@ -129,9 +129,9 @@ __device__ void gemm_mma(const GemmSmem<BN>& sm, uint32_t tmem_base, int num_til
       const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
       if (!mbar_wait(sm.tempty(buf), aph ^ 1u, sm.abort_flag())) return;
       tc_fence_after();
-      VITQ_TRACE_EV(2);  // mma: TMEM buffer free
+      VITQ_TRACE_EV(2, cnt);  // mma: TMEM buffer free
       if (!mbar_wait(sm.full(stage), phase, sm.abort_flag())) return;
-      VITQ_TRACE_EV(3);  // mma: operands landed
+      VITQ_TRACE_EV(3, cnt);  // mma: operands landed
       tc_fence_after();
       const uint32_t a0 = sm.a(stage), b0 = sm.b(stage);
 #pragma unroll
@@ -202,10 +202,10 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
         sw_next = col_ok ? __ldg(sw_ptr + kb + 1) : 0.f;
       }
       const uint64_t s2 = pack2(scale, scale);
-      if (lane == 0) VITQ_TRACE_EV(4);  // epilogue: waiting for partial
+      if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(4, cnt);  // epilogue: waiting for partial
       const bool ok = mbar_wait(sm.tfull(buf), aph, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
-      if (lane == 0) VITQ_TRACE_EV(5);  // epilogue: partial ready
+      if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(5, cnt);  // epilogue: partial ready
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + cg * 128;
 #pragma unroll
@@ -224,7 +224,7 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) VITQ_TRACE_EV(6);  // epilogue: partial consumed
+      if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(6, cnt);  // epilogue: partial consumed
       if (lane == 0) mbar_arrive(sm.tempty(buf));
     }
     if (row_ok && col_ok) {

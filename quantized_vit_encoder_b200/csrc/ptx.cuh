@@ -16,27 +16,27 @@ __device__ unsigned int g_device_error = 0;
 constexpr unsigned int kErrWaitTimeout = 1u;
 // A wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+// Longest single sleep inside a bounded wait (the abort flag and the limit are
+// checked between sleeps).
+constexpr uint32_t kWaitSleepNs = 100000u;
 
-// Event tracing for development builds (-DVITQ_TRACE): records (clock64, tag,
-// warp) for CTA 0 into a device buffer read by vitq_trace_read.  Compiles to
-// nothing in normal builds.
+// Event tracing for development builds (-DVITQ_TRACE): CTA 0 stores clock64()
+// for event `tag` at index `idx` (a loop count of the recording thread) into a
+// device table read by vitq_trace_read.  A plain store, so the recording
+// thread does not wait.  Compiles to nothing in normal builds.
 #ifdef VITQ_TRACE
-constexpr unsigned kTraceCap = 1u << 16;
-__device__ unsigned long long g_trace[kTraceCap][2];
-__device__ unsigned int g_trace_n = 0;
-#define VITQ_TRACE_EV(tag)                                                        \
-  do {                                                                            \
-    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {                  \
-      unsigned i_ = atomicAdd(&g_trace_n, 1u);                                    \
-      if (i_ < kTraceCap) {                                                       \
-        g_trace[i_][0] = clock64();                                               \
-        g_trace[i_][1] = ((unsigned long long)(tag) << 16) | (threadIdx.x >> 5);  \
-      }                                                                           \
-    }                                                                             \
+constexpr unsigned kTraceTags = 32, kTracePerTag = 4096;
+__device__ unsigned long long g_trace[kTraceTags][kTracePerTag];
+#define VITQ_TRACE_EV(tag, idx)                                              \
+  do {                                                                       \
+    if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0) {             \
+      const unsigned i_ = (unsigned)(idx);                                   \
+      if (i_ < kTracePerTag) g_trace[(tag)][i_] = clock64();                 \
+    }                                                                        \
   } while (0)
 #else
-#define VITQ_TRACE_EV(tag) \
-  do {                     \
+#define VITQ_TRACE_EV(tag, idx) \
+  do {                          \
   } while (0)
 #endif
 
@@ -81,18 +81,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may sleep up to `ns` nanoseconds waiting for
+// the phase (it wakes when the phase completes), so a waiting warp does not take
+// issue slots from the warps that share its scheduler.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait for the phase of `bar` with the given parity to complete.  Returns false
 // (and raises the shared abort flag and the device error word) if it has not
 // completed within limit_ns, or if another warp of the CTA already aborted.
 __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                 unsigned long long limit_ns) {
-#pragma unroll 1
-  for (int i = 0; i < 32; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
 #pragma unroll 1
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
     if (*abort_flag) return false;
     if (globaltimer_ns() - t0 > limit_ns) {
       atomicOr(&g_device_error, kErrWaitTimeout);
