@@ -8,7 +8,12 @@
  * ---------------------------------
  *  - Pointers are DEVICE pointers unless a parameter says "host".  The caller
  *    owns all memory; the library never allocates, frees or synchronises the
- *    host (except vitq_get_device_error, which reads a device word).
+ *    host (except vitq_get_device_error, which reads a device word, and the
+ *    one-time setup below).
+ *  - The first call on each device that reaches the device checks its
+ *    architecture and fills the library's GELU table on that device (a 128 KB
+ *    array of the library, one kernel on a private stream, waited for).  Make
+ *    that first call before any stream capture begins.
  *  - bf16 tensors are passed as `const void*` / `void*` holding IEEE bfloat16
  *    values; FP8 codes are OCP E4M3 ("E4M3FN") bytes; scales are fp32.
  *  - Matrices are row-major.  Activation FP8 codes are [M, K] (K contiguous);
@@ -102,7 +107,9 @@ int vit_ln_quant(const void* x, int M, int K, int ldx, const void* gamma, const 
                  uint8_t* q, float* s, int lds, void* stream);
 
 /* GELU(tanh) of a bf16 activation, rounded to bf16, quantised as in
- * vit_quant_act ([FRT] s3 gelu_tanh_to_fp8_block128).  f: bf16 [M, ldf]. */
+ * vit_quant_act ([FRT] s3 gelu_tanh_to_fp8_block128).  f: bf16 [M, ldf].
+ * The bf16 GELU of each input is read from a table holding, for every bf16
+ * value, the bf16 rounding of the fp64 value x / (1 + exp(-2u)). */
 int vit_gelu_quant(const void* f, int M, int K, int ldf, uint8_t* q, float* s, int lds, void* stream);
 
 /* FP8 W8A8 block-scaled GEMM with fused bias and residual ([FRT] s1 "FP8
@@ -181,8 +188,9 @@ size_t vitq_merger_workspace_bytes(int n_tokens);
  *  - n_tokens > VITQ_MERGER_STATIC_MAX_TOKENS returns VITQ_ERR_WORKSPACE and
  *    launches nothing; other arguments as vit_merger_forward.
  *  - The first call on each device, with that device current, looks up the
- *    array's device address (and may load this library's kernels there).
- *    Make that first call before any stream capture begins.
+ *    array's device address (and may load this library's kernels there, and
+ *    does the one-time setup described at the top of this file).  Make that
+ *    first call before any stream capture begins.
  *  - All calls on one device share the array.  Calls issued in order on one
  *    stream are safe; calls that can overlap (different streams, or host
  *    threads, without ordering between them) race on it and corrupt each

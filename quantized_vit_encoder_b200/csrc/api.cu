@@ -61,6 +61,15 @@ int current_device_ok(int* num_sms) {
   if (d.checked == 0) {
     cudaDeviceProp p;
     if (cudaGetDeviceProperties(&p, dev) != cudaSuccess) return VITQ_ERR_CUDA;
+    if (p.major == 10 && p.minor == 0) {
+      // one-time setup: the GELU table of this device, built on a private stream
+      cudaStream_t s;
+      if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return VITQ_ERR_CUDA;
+      cudaError_t e = build_gelu_table(s);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+      cudaStreamDestroy(s);
+      if (e != cudaSuccess) return VITQ_ERR_CUDA;
+    }
     d.checked = (p.major == 10 && p.minor == 0) ? 1 : -1;
     d.num_sms = p.multiProcessorCount;
   }
@@ -242,7 +251,7 @@ int block_impl(const vitq_block_weights* w, __nv_bfloat16* x, int n, const int32
                    num_sms, st);
   if (r) return r;
   VITQ_LAUNCH("gelu_quant", st, 0, quant_bytes(dn, VITQ_MLP),
-              launch_gelu_quant(b.f, n, VITQ_MLP, VITQ_MLP, b.q, b.s, b.lds, st));
+              launch_gelu_quant(b.f, n, VITQ_MLP, VITQ_MLP, b.q, b.s, b.lds, num_sms, st));
   return gemm_checked(b.q, b.s, b.lds, w->fc2_q, w->fc2_s, w->fc2_b, b.x1, x, n, VITQ_HIDDEN, VITQ_MLP,
                       num_sms, st);
 }
@@ -258,7 +267,7 @@ int merger_impl(const vitq_merger_weights* w, const __nv_bfloat16* x, int n, __n
                        VITQ_MERGE_IN, num_sms, st);
   if (r) return r;
   VITQ_LAUNCH("gelu_quant", st, 0, quant_bytes(rows, VITQ_MERGE_IN),
-              launch_gelu_quant(m.h, rows, VITQ_MERGE_IN, VITQ_MERGE_IN, m.q, m.s, m.lds, st));
+              launch_gelu_quant(m.h, rows, VITQ_MERGE_IN, VITQ_MERGE_IN, m.q, m.s, m.lds, num_sms, st));
   return gemm_checked(m.q, m.s, m.lds, w->fc2_q, w->fc2_s, w->fc2_b, nullptr, out, rows, VITQ_OUT_HIDDEN,
                       VITQ_MERGE_IN, num_sms, st);
 }
@@ -338,9 +347,11 @@ int vit_gelu_quant(const void* f, int M, int K, int ldf, uint8_t* q, float* s, i
   VITQ_CHECK(M >= 0 && K > 0 && ldf >= K && lds >= M, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(K % 16 == 0 && ldf % 8 == 0, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(f) && al16(q), VITQ_ERR_ALIGN);
-  int r = current_device_ok(nullptr);
+  int sms = 0;
+  int r = current_device_ok(&sms);
   if (r) return r;
-  VITQ_LAUNCH("gelu_quant", S(stream), 0, quant_bytes(M, K), launch_gelu_quant((const __nv_bfloat16*)f, M, K, ldf, q, s, lds, S(stream)));
+  VITQ_LAUNCH("gelu_quant", S(stream), 0, quant_bytes(M, K),
+              launch_gelu_quant((const __nv_bfloat16*)f, M, K, ldf, q, s, lds, sms, S(stream)));
   return VITQ_OK;
 }
 

@@ -221,64 +221,64 @@ __global__ void ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
 
 // ------------------------------------------------------------- GELU + quant
 // GELU(tanh) = 0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)), u = sqrt(2/pi)(x + 0.044715 x^3).
-// The fp32 sigmoid form (hardware exp2 and reciprocal) has no cancellation; its
-// relative error is below 2^-21 (|u| + 2) (measured against fp64 over x in
-// [-12, 9]).  When the result lies within 2^-20 (|u| + 4) |g| of a bf16 rounding
-// midpoint (or is below 1e-30) it is recomputed in fp64, so the bf16 result is
-// the rounding of the fp64 value x / (1 + exp(-2u)).
+// Its input is a bf16 value (the rounded fc1 output), so the bf16 result is a
+// function of 16 bits: g_gelu_table holds it for every bf16 bit pattern,
+// evaluated once per device in fp64 (the sigmoid form does not cancel for
+// u << 0) and rounded to bf16.  The GELU pass is then one shared-memory lookup
+// per element followed by the block-128 quantisation.
 
-__device__ __forceinline__ float gelu_f64_bf16(float x) {
+__device__ uint16_t g_gelu_table[65536];
+
+__global__ void gelu_table_kernel() {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 65536) return;
+  const float x = __uint_as_float((uint32_t)i << 16);
   const double xd = (double)x;
   const double ud = 0.79788456080286535588 * (xd + 0.044715 * xd * xd * xd);
-  return __bfloat162float(__double2bfloat16(xd / (1.0 + exp(-2.0 * ud))));
+  const __nv_bfloat16 g = __double2bfloat16(xd / (1.0 + exp(-2.0 * ud)));
+  g_gelu_table[i] = *reinterpret_cast<const uint16_t*>(&g);
 }
 
-// fp32 GELU of 8 values rounded to bf16; returns true if any of them lies within
-// its error bound of a bf16 rounding midpoint (then gelu_f64_bf16 decides it).
-__device__ __forceinline__ bool gelu8_fast(const float (&x)[8], float (&g)[8], bool (&slow)[8]) {
-  bool any = false;
+constexpr int kGeluThreads = 1024;
+constexpr size_t kGeluSmem = 65536 * 2;
+
+// Persistent: one CTA per SM copies the table into shared memory, then each warp
+// takes (row, 256-column step) items in turn (lane layout of lane_col).
+__global__ void __launch_bounds__(kGeluThreads, 1)
+    gelu_quant_kernel(const __nv_bfloat16* __restrict__ f, int M, int K, int ldf,
+                      uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+  extern __shared__ __align__(16) uint16_t lut[];
+  {
+    const uint4* src = reinterpret_cast<const uint4*>(g_gelu_table);
+    uint4* dst = reinterpret_cast<uint4*>(lut);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float u = x[i] * fmaf(0.035677408136300125f, x[i] * x[i], 0.7978845608028654f);
-    float e, rc;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-2.8853900817779268f * u));   // exp(-2u)
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(rc) : "f"(1.0f + e));
-    const float gv = x[i] * rc;
-    const float gr = __bfloat162float(__float2bfloat16_rn(gv));
-    const float half = __uint_as_float((__float_as_uint(gv) & 0x7F800000u) - (8u << 23));
-    const float err = fabsf(gv) * (fabsf(u) + 4.0f) * 9.5367431640625e-07f;  // 2^-20 (|u| + 4) |g|
-    slow[i] = (half - fabsf(gv - gr) <= err) | (fabsf(gv) < 1e-30f);
-    any |= slow[i];
-    g[i] = gr;
+    for (int i = 0; i < 8; ++i) dst[threadIdx.x + i * kGeluThreads] = src[threadIdx.x + i * kGeluThreads];
   }
-  return any;
-}
-
-__global__ void gelu_quant_kernel(const __nv_bfloat16* __restrict__ f, int M, int K, int ldf,
-                                  uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+  __syncthreads();
   const int steps = (K + 255) / 256;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long items = (long long)M * steps;
   const int lane = threadIdx.x & 31;
-  if (warp >= M * steps) return;
-  const int row = warp / steps;
-  const int st = warp - row * steps;
-  const int col = lane_col(st, lane);
-  const bool ok = col < K;
-  float v[8];
-  if (ok) {
-    float xv[8];
-    bool slow[8];
-    load8_bf16(f + (size_t)row * ldf + col, xv);
-    if (gelu8_fast(xv, v, slow)) {
+  const long long warps = (long long)gridDim.x * (kGeluThreads / 32);
+  for (long long w = blockIdx.x * (kGeluThreads / 32) + (threadIdx.x >> 5); w < items; w += warps) {
+    const int row = (int)(w / steps);
+    const int st = (int)(w - (long long)row * steps);
+    const int col = lane_col(st, lane);
+    const bool ok = col < K;
+    float v[8];
+    if (ok) {
+      const uint4 u = *reinterpret_cast<const uint4*>(f + (size_t)row * ldf + col);
+      const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (slow[i]) v[i] = gelu_f64_bf16(xv[i]);
+      for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float((uint32_t)lut[wd[i] & 0xFFFFu] << 16);
+        v[2 * i + 1] = __uint_as_float((uint32_t)lut[wd[i] >> 16] << 16);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = 0.f;
     }
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    quant_store(v, ok, lane, row, col, K, q, s, lds);
   }
-  quant_store(v, ok, lane, row, col, K, q, s, lds);
 }
 
 // ------------------------------------------------------------ weight quant
@@ -520,13 +520,21 @@ cudaError_t launch_ln_quant(const __nv_bfloat16* x, int ldx, const __nv_bfloat16
   return cudaGetLastError();
 }
 
+cudaError_t build_gelu_table(cudaStream_t st) {
+  gelu_table_kernel<<<256, 256, 0, st>>>();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gelu_quant(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* q, float* s,
-                              int lds, cudaStream_t st) {
+                              int lds, int num_sms, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  const int threads = 256;
+  cudaError_t e = cudaFuncSetAttribute(gelu_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kGeluSmem);
+  if (e != cudaSuccess) return e;
   const long long warps = (long long)M * ((K + 255) / 256);
-  gelu_quant_kernel<<<(unsigned)((warps * 32 + threads - 1) / threads), threads, 0, st>>>(f, M, K, ldf,
-                                                                                         q, s, lds);
+  const long long ctas = (warps + kGeluThreads / 32 - 1) / (kGeluThreads / 32);
+  gelu_quant_kernel<<<(unsigned)(ctas < num_sms ? ctas : num_sms), kGeluThreads, kGeluSmem, st>>>(
+      f, M, K, ldf, q, s, lds);
   return cudaGetLastError();
 }
 

@@ -29,8 +29,10 @@ cudaError_t launch_quant_act(const __nv_bfloat16* x, int M, int K, int ldx, uint
 cudaError_t launch_ln_quant(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma,
                             const __nv_bfloat16* beta, int M, int K, double eps, uint8_t* q,
                             float* s, int lds, cudaStream_t st);
+// One-time per device: GELU of every bf16 value into the device table.
+cudaError_t build_gelu_table(cudaStream_t st);
 cudaError_t launch_gelu_quant(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* q, float* s,
-                              int lds, cudaStream_t st);
+                              int lds, int num_sms, cudaStream_t st);
 cudaError_t launch_quant_weight(const __nv_bfloat16* w, int N, int K, uint8_t* q, float* s,
                                 cudaStream_t st);
 cudaError_t launch_rope_table(const int32_t* pos, int n, double theta, float* cs, cudaStream_t st);

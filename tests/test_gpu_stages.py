@@ -142,6 +142,18 @@ def test_gelu_quant_wide_range_bands(lib):
     assert_codes_equal(q, s, qr, sr, "gelu wide")
 
 
+def test_gelu_quant_every_bf16_value(lib):
+    """All 65024 finite bf16 bit patterns, in pattern order (each group of 128 holds
+    neighbouring values of one sign), through GELU + quant against the oracle."""
+    from quantized_vit_encoder_b200 import vitq
+    pats = np.arange(65536, dtype=np.uint32)
+    pats = pats[((pats >> 7) & 0xFF) != 0xFF]                       # drop inf / NaN
+    f = torch.from_numpy((pats << 16).view(np.float32)).to(torch.bfloat16).reshape(-1, 256)
+    q, s = vitq.gelu_quant(f.cuda())
+    qr, sr = ov.gelu_quant(f64(f))
+    assert_codes_equal(q, s, qr, sr, "gelu every bf16")
+
+
 def test_ln_quant_offset_mean(lib):
     """Rows with |mean| several times their spread (the one-pass variance is still exact enough)."""
     from quantized_vit_encoder_b200 import vitq
