@@ -6,16 +6,17 @@
 // with cu_seqlens): O = softmax(Q K^T * scale) V per segment and head.
 //
 // Design (B200):
-//   * one CTA per (segment, head, 256 queries = two 128-row Q tiles); 12 warps:
-//     TMA producer, one MMA issuer per Q tile, and one softmax warpgroup per Q
-//     tile (thread = query row = TMEM lane).  S_x(j+1) is computed while the
-//     softmax of S_x(j) runs (the softmax frees S_x once it holds it in
-//     registers), and the two tiles interleave on the tensor core;
+//   * one CTA per (segment, head, 256 queries = two 128-row Q tiles); 20 warps:
+//     TMA producer, one MMA issuer per Q tile, and eight softmax warps per Q
+//     tile, two per TMEM lane quadrant (thread = query row = TMEM lane; each
+//     warp of a pair owns 64 of the tile's 128 score columns, and the pair
+//     combines its row maxima through shared memory).  S_x(j+1) is computed
+//     while the softmax of S_x(j) runs (the softmax frees S_x once it holds it
+//     in registers), and the two tiles interleave on the tensor core;
 //   * the softmax exponentials run on MUFU ex2; a share can move to a polynomial
-//     on the FMA pipe (kPolyEvery) to balance the two pipes.  The two softmax
-//     warps that share an SMSP (tile A and tile B) take turns for their
-//     exponentials, so each turn has MUFU to itself while the other warp reads
-//     its next scores and waits for its P.V;
+//     on the FMA pipe (kPolyEvery).  The softmax warps of tile A and tile B that
+//     share an SMSP take turns for their exponentials, so each turn has MUFU to
+//     itself while the other tile reads its next scores and waits for its P.V;
 //   * K and V are read straight from the packed qkv activation [n, 3, 16, 72]
 //     through 3D TMA maps (d, slot, token).  head_dim 72 is padded to 80 by
 //     the tensor map itself: d >= 72 lies outside the map so TMA fills zeros,
@@ -23,13 +24,13 @@
 //     d 64..79 in a 32B-swizzled tile.  V: d 0..63 and d 64..127 in two
 //     128B-swizzled tiles, so that P.V is one N = 80 MMA per 16 keys (two
 //     MMAs of N = 64 and 16 cost twice as much: each re-reads P);
-//   * each softmax thread copies its Q row into TMEM once (columns packed two
+//   * the softmax threads copy their Q rows into TMEM once (columns packed two
 //     bf16 per 32-bit column), and S = Q K^T runs as 5 tcgen05.mma with A in
 //     TMEM (K = 16 each) into the tile's TMEM S buffer;
 //   * the softmax warps keep a running max in the log2 domain and rescale O
-//     (in TMEM) only when the max grows by more than 8, write P as bf16 into a
-//     128B-swizzled shared tile, and the MMA warp accumulates O += P V with V
-//     as an MN-major operand (two MMAs: N = 64 and N = 16);
+//     (in TMEM) only when the max grows by more than 8, write P into a
+//     128B-swizzled shared tile, and the MMA thread accumulates O += P V with
+//     V as an MN-major operand;
 //   * the epilogue divides by the row sum and stores bf16 O at column h*72.
 #include "internal.h"
 #include "ptx.cuh"
@@ -45,11 +46,15 @@ constexpr int kKV0 = 0, kKVStride = 53248;
 constexpr int kKLo = 0, kKHi = 16384, kVLo = 20480, kVHi = 36864;   // V hi = V lo + 16384 (N-atom stride)
 constexpr int kP0 = kKV0 + kStages * kKVStride;         // P tile X: two 64-key atoms of 16 KB
 constexpr int kPBytes = 32768;
-constexpr int kBar = kP0 + kQTiles * kPBytes;
+// Row-maximum exchange of the two softmax warps of a row quadrant:
+// [tile][step parity][half][128 rows] fp32 (the last exchange carries the row sums).
+constexpr int kRed = kP0 + kQTiles * kPBytes;
+constexpr int kBar = kRed + kQTiles * 2 * 2 * 128 * 4;
 // barriers: slot 0 (unused), kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2],
-// s_free[2], turn[2][4] (softmax warp of tile x on SMSP q finished its
-// exponentials), q_ready[2] (Q tile x is in TMEM)
-constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles;
+// s_free[2], turn[2][4] (the softmax warps of tile x on SMSP q finished their
+// exponentials), q_ready[2] (Q tile x is in TMEM), pair[2][4] (both halves of
+// tile x, quadrant q, posted their partial row maxima)
+constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles + kQTiles * 4;
 constexpr size_t kAttnSmem = 1024 + kBar + kNumBars * 8 + 16;
 static_assert(kAttnSmem <= 232448, "shared memory budget");
 // TMEM columns: S_A 0..127, S_B 128..255, O_A 256..335, Q_A 336..383, O_B 384..463,
@@ -58,8 +63,9 @@ __device__ __forceinline__ uint32_t tmem_s(int x) { return (uint32_t)x * 128u; }
 __device__ __forceinline__ uint32_t tmem_o(int x) { return 256u + (uint32_t)x * 128u; }
 __device__ __forceinline__ uint32_t tmem_q(int x) { return 336u + (uint32_t)x * 128u; }
 // Warpgroup 0: warp 0 TMA producer, warps 1 and 2 MMA issuers for Q tiles A
-// and B (warp 3 idle); warpgroups 1 and 2: softmax of Q tiles A and B.
-constexpr int kThreads = 128 * (1 + kQTiles);
+// and B (warp 3 idle); warps 4-11 softmax of Q tile A, 12-19 of Q tile B (two
+// warps per TMEM lane quadrant, each owning 64 of the 128 score columns).
+constexpr int kThreads = 128 + 256 * kQTiles;
 // Share of the softmax exponentials moved from MUFU to the FMA-pipe polynomial:
 // one pair in kPolyEvery (0 = none).  MUFU ex2 runs at 16 per clock per SM.
 #ifndef VITQ_ATTN_POLY_EVERY
@@ -100,6 +106,12 @@ struct AttnSmem {
   __device__ uint32_t pv_done(int x) const { return smem_u32(bar(1 + 2 * kStages + 2 * kQTiles + x)); }
   __device__ uint32_t s_free(int x) const { return smem_u32(bar(1 + 2 * kStages + 3 * kQTiles + x)); }
   __device__ uint32_t turn(int x, int q) const { return smem_u32(bar(1 + 2 * kStages + 4 * kQTiles + x * 4 + q)); }
+  __device__ uint32_t pair(int x, int q) const {
+    return smem_u32(bar(1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles + x * 4 + q));
+  }
+  __device__ float* red(int x, int par, int h) const {
+    return reinterpret_cast<float*>(base + kRed) + ((x * 2 + par) * 2 + h) * 128;
+  }
   __device__ uint32_t* tmem_holder() const { return reinterpret_cast<uint32_t*>(bar(kNumBars)); }
   __device__ volatile int* abort_flag() const {
     return reinterpret_cast<volatile int*>(tmem_holder() + 1);
@@ -244,34 +256,40 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi, bool f16) {
   return pack_bf16x2(lo, hi);
 }
 
-// One warpgroup per Q tile; thread = query row = TMEM lane.  S is read from
-// TMEM twice (row max, then exponentials), 64 columns at a time, so a thread
-// holds at most 64 scores in registers.
+// Two warps per (Q tile, TMEM lane quadrant); thread = query row = TMEM lane.
+// Half h of the pair owns score columns 64h..64h+63 of its rows and P atom h.
+// The halves combine their row maxima through shared memory every step (so
+// both follow the same running max); the row sums stay partial until the end.
+// Half 0 also copies the Q rows into TMEM, rescales O and writes the output.
 template <bool kVF16>
-__device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& g, int x, int n_q, int head,
-                             int seq_start, int seq_len, int q0, int n_kv, int off) {
+__device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& g, int x, int h, int n_q,
+                             int head, int seq_start, int seq_len, int q0, int n_kv, int off) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;
   const int r = quad * 32 + lane;
   const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-  const uint32_t s_addr = tmem + lane_addr + tmem_s(x), o_addr = tmem + lane_addr + tmem_o(x);
-  uint8_t* pbase = sm.base + kP0 + x * kPBytes;
-  {
+  const uint32_t s_addr = tmem + lane_addr + tmem_s(x) + 64 * h, o_addr = tmem + lane_addr + tmem_o(x);
+  uint8_t* pbase = sm.base + kP0 + x * kPBytes + h * 16384;
+  const bool tr = h == 0 && quad == 0 && lane == 0;
+  (void)tr;
+  if (h == 0) {
     // this thread's Q row -> TMEM (bf16 pairs in columns 0..35, zeros up to 47)
-    uint32_t qw[3][16];
     const bool q_ok = q0 + r < seq_len && seq_start + q0 + r < g.n_tokens;
     const uint4* src = reinterpret_cast<const uint4*>(g.qkv + (size_t)(seq_start + q0 + r) * 3456 + head * 72);
-#pragma unroll
-    for (int i = 0; i < 12; ++i) {
-      const uint4 v = (q_ok && i < 9) ? __ldg(src + i) : make_uint4(0u, 0u, 0u, 0u);
-      qw[i >> 2][(i & 3) * 4 + 0] = v.x;
-      qw[i >> 2][(i & 3) * 4 + 1] = v.y;
-      qw[i >> 2][(i & 3) * 4 + 2] = v.z;
-      qw[i >> 2][(i & 3) * 4 + 3] = v.w;
-    }
     const uint32_t q_addr = tmem + lane_addr + tmem_q(x);
 #pragma unroll
-    for (int c = 0; c < 3; ++c) tmem_st16(q_addr + c * 16, qw[c]);
+    for (int c = 0; c < 3; ++c) {
+      uint32_t qw[16];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = (q_ok && c * 4 + i < 9) ? __ldg(src + c * 4 + i) : make_uint4(0u, 0u, 0u, 0u);
+        qw[i * 4 + 0] = v.x;
+        qw[i * 4 + 1] = v.y;
+        qw[i * 4 + 2] = v.z;
+        qw[i * 4 + 3] = v.w;
+      }
+      tmem_st16(q_addr + c * 16, qw);
+    }
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
@@ -281,44 +299,51 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
   for (int j = 0; j < n_kv; ++j) {
     bool ok = mbar_wait(sm.s_full(x), (uint32_t)j & 1u, sm.abort_flag());
     if (!__all_sync(0xffffffffu, ok)) return;
-    if (lane == 0 && quad == 0) VITQ_TRACE_EV(20 + x, j);   // softmax: S ready
+    if (tr) VITQ_TRACE_EV(20 + x, j);   // softmax: S ready
     tc_fence_after();
-    const int valid = seq_len - kv_tile(j, off, n_kv) * kBN;   // keys of this tile inside the segment
-    // one TMEM round trip: all 128 scores of the row, then S_x is free for S_x(j+1)
-    uint32_t su[4][32];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld32(s_addr + c * 32, su[c]);
+    // keys of this tile inside the segment, counted from this half's first column
+    const int valid = seq_len - kv_tile(j, off, n_kv) * kBN - 64 * h;
+    uint32_t su[2][32];
+    tmem_ld32(s_addr, su[0]);
+    tmem_ld32(s_addr + 32, su[1]);
     tmem_wait_ld();
-    if (lane == 0 && quad == 0) VITQ_TRACE_EV(26 + x, j);   // softmax: S in registers
+    if (tr) VITQ_TRACE_EV(26 + x, j);   // softmax: S in registers
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.s_free(x));
-    if (valid < kBN) {
+    if (valid < 64) {
 #pragma unroll
-      for (int i = 0; i < 128; ++i)
+      for (int i = 0; i < 64; ++i)
         if (i >= valid) su[i >> 5][i & 31] = 0xFF800000u;   // -inf
     }
-    // row max: 8 independent chains of 3-input max, then a tree
+    // partial row max: 8 independent chains of 3-input max, then a tree
     float mp[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) mp[k] = __uint_as_float(su[0][k]);
 #pragma unroll
-    for (int i = 8; i < 128; i += 16)
+    for (int i = 8; i < 64; i += 16)
 #pragma unroll
       for (int k = 0; k < 8; ++k)
         mp[k] = fmax3(mp[k], __uint_as_float(su[(i + k) >> 5][(i + k) & 31]),
                       __uint_as_float(su[(i + 8 + k) >> 5][(i + 8 + k) & 31]));
-    const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) *
-                     g.scale_log2;
+    const float pm = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
+    sm.red(x, j & 1, h)[r] = pm;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.pair(x, quad));
+    ok = mbar_wait(sm.pair(x, quad), (uint32_t)j & 1u, sm.abort_flag());
+    if (!__all_sync(0xffffffffu, ok)) return;
+    const float mx = fmaxf(pm, sm.red(x, j & 1, 1 - h)[r]) * g.scale_log2;
     if (j > 0) {
+      // P(j) overwrites P(j-1), and half 0 may rescale O: P(j-1).V must be done
       ok = mbar_wait(sm.pv_done(x), (uint32_t)(j - 1) & 1u, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
       tc_fence_after();
     }
-    if (lane == 0 && quad == 0) VITQ_TRACE_EV(22 + x, j);   // softmax: max known, O stable
+    if (tr) VITQ_TRACE_EV(22 + x, j);   // softmax: max known, O stable
     // new running max: it changes only when the tile max exceeds it by more than 8
     // (so P <= 2^8), and the decision is warp-uniform because the O rescale uses
     // warp-collective tcgen05.ld/st (rows that keep their max get alpha = 1).
+    // Both halves see the same maxima, so they take the same decisions.
     float alpha = 1.f;
     bool rescale = false;
     if (j == 0) {
@@ -331,59 +356,55 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
         m_run = mx;
       }
     }
-    // The two tiles' softmax warps on one SMSP take turns for the exponentials
-    // (A(j), B(j), A(j+1), ...): MUFU runs one tile at full rate while the other
-    // tile loads its scores, takes the row max and waits for its P.V.
+    // The softmax warps of the two tiles on one SMSP take turns for the
+    // exponentials (A(j), B(j), A(j+1), ...): MUFU serves one tile at full rate
+    // while the other reads its next scores and waits for its P.V.
     if (n_q == 2 && (x == 1 || j > 0)) {
       ok = mbar_wait(sm.turn(1 - x, quad), (uint32_t)(x == 1 ? j : j - 1) & 1u, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
     }
-    if (lane == 0 && quad == 0) VITQ_TRACE_EV(28 + x, j);   // softmax: turn for the exponentials
-    // P = 2^(s * scale_log2 - m_run), rounded to the P.V operand type, into the swizzled
-    // P tile (64-key atom a holds keys 64a..64a+63); 8 fp32 partial row sums.
+    if (tr) VITQ_TRACE_EV(28 + x, j);   // softmax: turn for the exponentials
+    // P = 2^(s * scale_log2 - m_run), rounded to the P.V operand type, into this
+    // half's 64-key atom of the swizzled P tile; 8 fp32 partial row sums.
     const uint64_t sc2 = f2pack(g.scale_log2, g.scale_log2), nm2 = f2pack(-m_run, -m_run);
     uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-    for (int a = 0; a < 2; ++a) {
+    for (int c = 0; c < 8; ++c) {
+      uint32_t w[4];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int k0 = a * 64 + c * 8 + 2 * i;
-          const float2 t = f2unpack(ffma2(f2pack(__uint_as_float(su[k0 >> 5][k0 & 31]),
-                                                 __uint_as_float(su[(k0 + 1) >> 5][(k0 + 1) & 31])),
-                                          sc2, nm2));
-          // every kPolyEvery-th pair runs the FMA-pipe polynomial, the rest MUFU ex2
-          float2 p;
-          if (kPolyEvery > 0 && (i % kPolyMod) == kPolyMod - 1) {
-            p = ex2_poly2(t.x, t.y);
-          } else {
-            p.x = ex2(t.x);
-            p.y = ex2(t.y);
-          }
-          w[i] = pack_p(p.x, p.y, kVF16);
-          ls[i] = fadd2(ls[i], f2pack(p.x, p.y));
+      for (int i = 0; i < 4; ++i) {
+        const int k0 = c * 8 + 2 * i;
+        const float2 t = f2unpack(ffma2(f2pack(__uint_as_float(su[k0 >> 5][k0 & 31]),
+                                               __uint_as_float(su[(k0 + 1) >> 5][(k0 + 1) & 31])),
+                                        sc2, nm2));
+        // every kPolyEvery-th pair runs the FMA-pipe polynomial, the rest MUFU ex2
+        float2 p;
+        if (kPolyEvery > 0 && (i % kPolyMod) == kPolyMod - 1) {
+          p = ex2_poly2(t.x, t.y);
+        } else {
+          p.x = ex2(t.x);
+          p.y = ex2(t.y);
         }
-        uint8_t* dst = pbase + a * 16384 + r * 128 + ((c ^ (r & 7)) << 4);
-        *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        w[i] = pack_p(p.x, p.y, kVF16);
+        ls[i] = fadd2(ls[i], f2pack(p.x, p.y));
       }
+      uint8_t* dst = pbase + r * 128 + ((c ^ (r & 7)) << 4);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (n_q == 2 && !(x == 1 && j == n_kv - 1)) {   // hand the turn to the other tile
       __syncwarp();
       if (lane == 0) mbar_arrive(sm.turn(x, quad));
     }
-    if (rescale) {
+    if (rescale && h == 0) {
       // O (complete up to P.V(j-1)) to the new max; done after P so the scores are dead
-      uint32_t u[5][16];
-#pragma unroll
-      for (int c = 0; c < 5; ++c) tmem_ld16(o_addr + c * 16, u[c]);
-      tmem_wait_ld();
-#pragma unroll
+#pragma unroll 1
       for (int c = 0; c < 5; ++c) {
+        uint32_t u[16];
+        tmem_ld16(o_addr + c * 16, u);
+        tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) u[c][i] = __float_as_uint(__uint_as_float(u[c][i]) * alpha);
-        tmem_st16(o_addr + c * 16, u[c]);
+        for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(__uint_as_float(u[i]) * alpha);
+        tmem_st16(o_addr + c * 16, u);
       }
       tmem_wait_st();
     }
@@ -394,30 +415,39 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0 && quad == 0) VITQ_TRACE_EV(24 + x, j);   // softmax: P written
+    if (tr) VITQ_TRACE_EV(24 + x, j);   // softmax: P written
     if (lane == 0) mbar_arrive(sm.p_full(x));
   }
   bool ok = mbar_wait(sm.pv_done(x), (uint32_t)(n_kv - 1) & 1u, sm.abort_flag());
   if (!__all_sync(0xffffffffu, ok)) return;
   tc_fence_after();
+  // row sum = the two halves' partial sums (one more exchange, slot parity n_kv)
+  sm.red(x, n_kv & 1, h)[r] = l_run;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(sm.pair(x, quad));
+  ok = mbar_wait(sm.pair(x, quad), (uint32_t)n_kv & 1u, sm.abort_flag());
+  if (!__all_sync(0xffffffffu, ok)) return;
+  if (h != 0) return;
+  const float l_sum = l_run + sm.red(x, n_kv & 1, 1)[r];
   // O / l in 16-column chunks (columns 72..79 are the zero padding and are not stored)
   const bool row_ok = q0 + r < seq_len && seq_start + q0 + r < g.n_tokens;
-  const float inv = 1.0f / l_run;
+  const float inv = 1.0f / l_sum;
   __nv_bfloat16* dst = g.out + (size_t)(seq_start + q0 + r) * 1152 + head * 72;
-  uint32_t u[5][16];
 #pragma unroll
-  for (int c = 0; c < 5; ++c) tmem_ld16(o_addr + c * 16, u[c]);
-  tmem_wait_ld();
-  if (row_ok) {
+  for (int c = 0; c < 5; ++c) {
+    uint32_t u[16];
+    tmem_ld16(o_addr + c * 16, u);
+    tmem_wait_ld();
 #pragma unroll
-    for (int c8 = 0; c8 < 9; ++c8) {
-      const int c = c8 >> 1, h = c8 & 1;
-      uint4 v;
-      v.x = pack_bf16x2(__uint_as_float(u[c][h * 8 + 0]) * inv, __uint_as_float(u[c][h * 8 + 1]) * inv);
-      v.y = pack_bf16x2(__uint_as_float(u[c][h * 8 + 2]) * inv, __uint_as_float(u[c][h * 8 + 3]) * inv);
-      v.z = pack_bf16x2(__uint_as_float(u[c][h * 8 + 4]) * inv, __uint_as_float(u[c][h * 8 + 5]) * inv);
-      v.w = pack_bf16x2(__uint_as_float(u[c][h * 8 + 6]) * inv, __uint_as_float(u[c][h * 8 + 7]) * inv);
-      *reinterpret_cast<uint4*>(dst + c8 * 8) = v;
+    for (int hh = 0; hh < 2; ++hh) {
+      if (row_ok && c * 2 + hh < 9) {
+        uint4 v;
+        v.x = pack_bf16x2(__uint_as_float(u[hh * 8 + 0]) * inv, __uint_as_float(u[hh * 8 + 1]) * inv);
+        v.y = pack_bf16x2(__uint_as_float(u[hh * 8 + 2]) * inv, __uint_as_float(u[hh * 8 + 3]) * inv);
+        v.z = pack_bf16x2(__uint_as_float(u[hh * 8 + 4]) * inv, __uint_as_float(u[hh * 8 + 5]) * inv);
+        v.w = pack_bf16x2(__uint_as_float(u[hh * 8 + 6]) * inv, __uint_as_float(u[hh * 8 + 7]) * inv);
+        *reinterpret_cast<uint4*>(dst + (c * 2 + hh) * 8) = v;
+      }
     }
   }
 }
@@ -444,12 +474,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(sm.kv_empty(s), (uint32_t)n_q);       // one commit per active Q tile
     }
     for (int x = 0; x < kQTiles; ++x) {
-      for (int q = 0; q < 4; ++q) mbar_init(sm.turn(x, q), 1);
+      for (int q = 0; q < 4; ++q) mbar_init(sm.turn(x, q), 2);
+      for (int q = 0; q < 4; ++q) mbar_init(sm.pair(x, q), 2);
       mbar_init(sm.q_ready(x), 4);
       mbar_init(sm.s_full(x), 1);
-      mbar_init(sm.p_full(x), 4);
+      mbar_init(sm.p_full(x), 8);
       mbar_init(sm.pv_done(x), 1);
-      mbar_init(sm.s_free(x), 4);
+      mbar_init(sm.s_free(x), 8);
     }
     *sm.abort_flag() = 0;
     fence_barrier_init();
@@ -471,8 +502,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       attn_mma<kVF16>(sm, tmem, warp - 1, n_kv);
     }
   } else {
-    const int x = (warp >> 2) - 1;
-    if (x < n_q) attn_softmax<kVF16>(sm, tmem, args, x, n_q, head, seq_start, seq_len, q0 + x * kBM, n_kv, off);
+    const int x = (warp - 4) >> 3, h = ((warp - 4) >> 2) & 1;
+    if (x < n_q)
+      attn_softmax<kVF16>(sm, tmem, args, x, h, n_q, head, seq_start, seq_len, q0 + x * kBM, n_kv, off);
   }
   tc_fence_before();
   __syncthreads();

@@ -123,18 +123,28 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ x, int M, int
 }
 
 // --------------------------------------------------------- LayerNorm + quant
-// One warp per row held in registers.  The statistics are exact fp64 sums of
-// the bf16 inputs (sum and sum of squares); the normalised value is evaluated
-// in fp32 and, when it lies within its error bound of a bf16 rounding
-// midpoint, recomputed in fp64, so the bf16 result is the rounding of the fp64
-// value (x - mean) * rstd * gamma + beta.
+// One warp per row, eight rows per CTA; gamma and beta are staged once per CTA
+// in shared memory.  The statistics are exact fp64 sums of the bf16 inputs
+// (sum and sum of squares); the normalised value is evaluated in fp32 and,
+// when it lies within its error bound of a bf16 rounding midpoint, recomputed
+// in fp64, so the bf16 result is the rounding of the fp64 value
+// (x - mean) * rstd * gamma + beta.
+
+constexpr int kLnRows = 8;
 
 template <int ITERS>
-__global__ void ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
-                                const __nv_bfloat16* __restrict__ gamma,
-                                const __nv_bfloat16* __restrict__ beta, int M, int K, double eps,
-                                uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
-  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+__global__ void __launch_bounds__(32 * kLnRows, 3)
+    ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx, const __nv_bfloat16* __restrict__ gamma,
+                    const __nv_bfloat16* __restrict__ beta, int M, int K, double eps,
+                    uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+  __shared__ uint4 sg[ITERS * 32], sb[ITERS * 32];
+  for (int i = threadIdx.x; i < ITERS * 32; i += blockDim.x) {
+    const int col = lane_col(i >> 5, i & 31);
+    sg[i] = col < K ? *reinterpret_cast<const uint4*>(gamma + col) : make_uint4(0, 0, 0, 0);
+    sb[i] = col < K ? *reinterpret_cast<const uint4*>(beta + col) : make_uint4(0, 0, 0, 0);
+  }
+  __syncthreads();
+  const int row = blockIdx.x * kLnRows + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
   // Rows of up to 8 steps stay in registers; wider rows (the merger's 4608) are
@@ -151,8 +161,8 @@ __global__ void ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
 #pragma unroll
     for (int it = 0; it < kHeld; ++it) raw[it] = load_step(it);
   }
-  // exact fp64 sums of the bf16 inputs (bf16 -> fp32 -> fp64 is exact); 4 chains each
-  double s1[4] = {0.0, 0.0, 0.0, 0.0}, s2[4] = {0.0, 0.0, 0.0, 0.0};
+  // exact fp64 sums of the bf16 inputs (bf16 -> fp32 -> fp64 is exact); 2 chains each
+  double s1[2] = {0.0, 0.0}, s2[2] = {0.0, 0.0};
 #pragma unroll
   for (int it = 0; it < ITERS; ++it) {
     float v[8];
@@ -160,11 +170,11 @@ __global__ void ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const double d = (double)v[i];
-      s1[i & 3] += d;
-      s2[i & 3] = fma(d, d, s2[i & 3]);
+      s1[i & 1] += d;
+      s2[i & 1] = fma(d, d, s2[i & 1]);
     }
   }
-  double t1 = (s1[0] + s1[1]) + (s1[2] + s1[3]), t2 = (s2[0] + s2[1]) + (s2[2] + s2[3]);
+  double t1 = s1[0] + s1[1], t2 = s2[0] + s2[1];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     t1 += __shfl_xor_sync(0xffffffffu, t1, o);
@@ -183,32 +193,34 @@ __global__ void ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx,
     unpack8(rv, v);
     if (ok) {
       float g[8], b[8];
-      load8_bf16(gamma + col, g);
-      load8_bf16(beta + col, b);
+      unpack8(sg[it * 32 + lane], g);
+      unpack8(sb[it * 32 + lane], b);
       bool slow = false;
-      float t[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        t[i] = ((v[i] - mh) - ml) * r32;
-        const float y = fmaf(t[i], g[i], b[i]);
+        const float t = ((v[i] - mh) - ml) * r32;
+        const float y = fmaf(t, g[i], b[i]);
         // fp32 error of y is below (|t g| + |b|) 2^-20; distance of y to the nearest
         // bf16 rounding midpoint = half a bf16 ulp (from y's exponent) - |y - bf16(y)|
         const float yr = __bfloat162float(__float2bfloat16_rn(y));
         const float half = __uint_as_float((__float_as_uint(y) & 0x7F800000u) - (8u << 23));
-        const float err = (fabsf(t[i] * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;
+        const float err = (fabsf(t * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;
         slow |= (half - fabsf(y - yr) <= err) | (fabsf(y) < 1e-30f);
         v[i] = yr;
       }
-      if (slow) {
-#pragma unroll
+      if (slow) {   // rare: redo the flagged values in fp64 from the inputs
+        float xi[8];
+        unpack8(rv, xi);
+        unpack8(sg[it * 32 + lane], g);
+        unpack8(sb[it * 32 + lane], b);
+#pragma unroll 1
         for (int i = 0; i < 8; ++i) {
-          const float y = fmaf(t[i], g[i], b[i]);
+          const float t = ((xi[i] - mh) - ml) * r32;
+          const float y = fmaf(t, g[i], b[i]);
           const float yr = __bfloat162float(__float2bfloat16_rn(y));
           const float half = __uint_as_float((__float_as_uint(y) & 0x7F800000u) - (8u << 23));
-          const float err = (fabsf(t[i] * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;
+          const float err = (fabsf(t * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;
           if (half - fabsf(y - yr) <= err || fabsf(y) < 1e-30f) {
-            float xi[8];
-            unpack8(rv, xi);
             const double yd = ((double)xi[i] - mean) * rstd * (double)g[i] + (double)b[i];
             v[i] = __bfloat162float(__double2bfloat16(yd));
           }
@@ -497,8 +509,7 @@ template <int IT>
 static void ln_launch(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* g,
                       const __nv_bfloat16* b, int M, int K, double eps, uint8_t* q, float* s, int lds,
                       cudaStream_t st) {
-  const int threads = 128;
-  ln_quant_kernel<IT><<<(unsigned)(((long long)M * 32 + threads - 1) / threads), threads, 0, st>>>(
+  ln_quant_kernel<IT><<<(unsigned)((M + kLnRows - 1) / kLnRows), 32 * kLnRows, 0, st>>>(
       x, ldx, g, b, M, K, eps, q, s, lds);
 }
 
