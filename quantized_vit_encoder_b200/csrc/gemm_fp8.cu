@@ -16,7 +16,12 @@
 //     reads the K block's partial from TMEM and accumulates
 //     acc += partial * sA * sW in registers (the scales differ per K block, so
 //     the tensor core cannot accumulate across K blocks); after the last K
-//     block it adds bias and residual and stores bf16.
+//     block it adds bias and residual and writes bf16 into the warp's
+//     128B-swizzled staging tile (32 rows x 128 columns), which one lane sends
+//     to global memory with TMA stores.  The residual tile arrives by TMA into
+//     the same staging tile while the K loop runs.  Row-per-thread global
+//     stores (each a separate 16-byte sector) used to stall the next tile's
+//     K loop for longer than the K loop itself.
 #include "internal.h"
 #include "ptx.cuh"
 
@@ -29,7 +34,7 @@ namespace {
 template <int BN>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 128;
-  static constexpr int STAGES = BN == 256 ? 4 : 6;
+  static constexpr int STAGES = BN == 256 ? 3 : 5;
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = BN * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -39,8 +44,10 @@ struct GemmCfg {
   static constexpr int THREADS = BN == 256 ? 384 : 192;
   static constexpr bool SPLIT_REGS = BN == 256;
   static constexpr int MIN_LAUNCH_REGS = 168;   // 384 x 168 >= 128 x 56 + 256 x 224 (BN = 256)
-  static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF) * 8 + 16;
-  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
+  static constexpr int OUT_WARP_BYTES = 2 * 4096;   // two 64-column SW128 boxes of 32 rows
+  static constexpr int OUT_BYTES = EPI_WARPS * OUT_WARP_BYTES;
+  static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF + EPI_WARPS) * 8 + 16;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + OUT_BYTES + 1024 + BAR_BYTES;
 };
 static_assert(384 * GemmCfg<256>::MIN_LAUNCH_REGS >= 128 * 56 + 256 * 224, "register split");
 
@@ -62,8 +69,11 @@ struct GemmSmem {
   __device__ uint32_t b(int s) const {
     return smem_u32(base + (size_t)s * Cfg::STAGE_BYTES + Cfg::A_BYTES);
   }
+  __device__ uint8_t* out(int w) const {
+    return base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + (size_t)w * Cfg::OUT_WARP_BYTES;
+  }
   __device__ uint64_t* bars() const {
-    return reinterpret_cast<uint64_t*>(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES);
+    return reinterpret_cast<uint64_t*>(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES);
   }
   __device__ uint32_t full(int s) const { return smem_u32(bars() + s); }
   __device__ uint32_t empty(int s) const { return smem_u32(bars() + Cfg::STAGES + s); }
@@ -71,8 +81,9 @@ struct GemmSmem {
   __device__ uint32_t tempty(int b) const {
     return smem_u32(bars() + 2 * Cfg::STAGES + Cfg::NBUF + b);
   }
+  __device__ uint32_t res_full(int w) const { return smem_u32(bars() + 2 * Cfg::STAGES + 2 * Cfg::NBUF + w); }
   __device__ uint32_t* tmem_holder() const {
-    return reinterpret_cast<uint32_t*>(bars() + 2 * Cfg::STAGES + 2 * Cfg::NBUF);
+    return reinterpret_cast<uint32_t*>(bars() + 2 * Cfg::STAGES + 2 * Cfg::NBUF + Cfg::EPI_WARPS);
   }
   __device__ volatile int* abort_flag() const {
     return reinterpret_cast<volatile int*>(tmem_holder() + 1);
@@ -169,22 +180,39 @@ __device__ __forceinline__ uint64_t fma2(uint64_t p, uint64_t s, uint64_t acc) {
 
 template <int BN>
 __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const GemmArgs& g,
-                              int tiles_m, int tiles_n, int num_tiles, int nkb) {
+                              const CUtensorMap* tmC, const CUtensorMap* tmR, int tiles_m, int tiles_n,
+                              int num_tiles, int nkb) {
   using Cfg = GemmCfg<BN>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;                         // TMEM lane quadrant this warp may access
-  const int cg = (warp - Cfg::EPI_WARP0) >> 2;       // which 128-column group of the tile
+  const int ew = warp - Cfg::EPI_WARP0;              // epilogue warp index
+  const int cg = ew >> 2;                            // which 128-column group of the tile
   const int r_in = quad * 32 + lane;
-  uint32_t cnt = 0;
-  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+  uint8_t* stg = sm.out(ew);                         // staging: [2 boxes][32 rows][128 B], SW128
+  const uint32_t stg_u32 = smem_u32(stg);
+  const bool has_res = g.residual != nullptr;
+  uint32_t cnt = 0, it = 0;
+  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
     int mt, nt;
     tile_coords(tile, tiles_m, tiles_n, mt, nt);
     const int m0 = mt * Cfg::BM;
     const int n0 = nt * BN;
     const int row = m0 + r_in;
     const int col0 = n0 + cg * 128;
+    const int y0 = m0 + quad * 32;                   // first row of this warp's staging tile
     const bool row_ok = row < g.M;
     const bool col_ok = col0 < g.N;
+    // the staging tile is free once the previous tile's stores have read it;
+    // then the residual tile (if any) is fetched into it during the K loop
+    if (lane == 0) {
+      bulk_wait_read_all();
+      if (has_res) {
+        mbar_arrive_expect_tx(sm.res_full(ew), Cfg::OUT_WARP_BYTES);
+        tma_load_2d(stg_u32, tmR, col0, y0, sm.res_full(ew));
+        tma_load_2d(stg_u32 + 4096, tmR, col0 + 64, y0, sm.res_full(ew));
+      }
+    }
+    __syncwarp();
     const float* sa_ptr = g.sA + row;
     const float* sw_ptr = g.sW + (size_t)(col0 >> 7) * nkb;
     uint64_t acc[64];
@@ -227,55 +255,72 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
       if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(6, cnt);  // epilogue: partial consumed
       if (lane == 0) mbar_arrive(sm.tempty(buf));
     }
-    if (row_ok && col_ok) {
-      __nv_bfloat16* crow = g.C + (size_t)row * g.N;
-      const __nv_bfloat16* rrow = g.residual ? g.residual + (size_t)row * g.N : nullptr;
+    if (has_res) {
+      const bool ok = mbar_wait(sm.res_full(ew), it & 1u, sm.abort_flag());
+      if (!__all_sync(0xffffffffu, ok)) return;
+    }
+    // bias + residual, bf16, into the staging tile (row = lane, 16-byte chunk c of
+    // box h at position c ^ (lane & 7))
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const int c8 = h * 8 + c;
         const int col = col0 + c8 * 8;
-        if (col < g.N) {
-          float v[8];
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float2 f = unpack2(acc[c8 * 4 + i]);
+          v[2 * i] = f.x;
+          v[2 * i + 1] = f.y;
+        }
+        if (g.bias && col < g.N) {
+          const uint4 bu = __ldg(reinterpret_cast<const uint4*>(g.bias + col));
+          const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float2 f = unpack2(acc[c8 * 4 + i]);
-            v[2 * i] = f.x;
-            v[2 * i + 1] = f.y;
+            const float2 f = unpack_bf16x2(bw[i]);
+            v[2 * i] += f.x;
+            v[2 * i + 1] += f.y;
           }
-          if (g.bias) {
-            const uint4 bu = __ldg(reinterpret_cast<const uint4*>(g.bias + col));
-            const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f = unpack_bf16x2(bw[i]);
-              v[2 * i] += f.x;
-              v[2 * i + 1] += f.y;
-            }
-          }
-          if (rrow) {
-            const uint4 ru = *reinterpret_cast<const uint4*>(rrow + col);
-            const uint32_t rw[4] = {ru.x, ru.y, ru.z, ru.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const float2 f = unpack_bf16x2(rw[i]);
-              v[2 * i] += f.x;
-              v[2 * i + 1] += f.y;
-            }
-          }
-          uint4 o;
-          o.x = pack_bf16x2(v[0], v[1]);
-          o.y = pack_bf16x2(v[2], v[3]);
-          o.z = pack_bf16x2(v[4], v[5]);
-          o.w = pack_bf16x2(v[6], v[7]);
-          *reinterpret_cast<uint4*>(crow + col) = o;
         }
+        uint4* slot = reinterpret_cast<uint4*>(stg + h * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4));
+        if (has_res) {
+          const uint4 ru = *slot;
+          const uint32_t rw[4] = {ru.x, ru.y, ru.z, ru.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 f = unpack_bf16x2(rw[i]);
+            v[2 * i] += f.x;
+            v[2 * i + 1] += f.y;
+          }
+        }
+        uint4 o;
+        o.x = pack_bf16x2(v[0], v[1]);
+        o.y = pack_bf16x2(v[2], v[3]);
+        o.z = pack_bf16x2(v[4], v[5]);
+        o.w = pack_bf16x2(v[6], v[7]);
+        *slot = o;
       }
     }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      // TMA clips rows >= M and columns >= N; boxes wholly outside are skipped
+      if (y0 < g.M) {
+        if (col0 < g.N) tma_store_2d(tmC, stg_u32, col0, y0);
+        if (col0 + 64 < g.N) tma_store_2d(tmC, stg_u32 + 4096, col0 + 64, y0);
+      }
+      bulk_commit_group();
+    }
   }
+  if (lane == 0) bulk_wait_all();
 }
 
 template <int BN>
 __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmR,
                     const GemmArgs args) {
   using Cfg = GemmCfg<BN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -296,6 +341,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
       mbar_init(sm.tfull(b), 1);
       mbar_init(sm.tempty(b), Cfg::EPI_WARPS);
     }
+    for (int w = 0; w < Cfg::EPI_WARPS; ++w) mbar_init(sm.res_full(w), 1);
     *sm.abort_flag() = 0;
     fence_barrier_init();
   }
@@ -319,7 +365,7 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     }
   } else {
     if (Cfg::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
-    gemm_epilogue<BN>(sm, tmem_base, args, tiles_m, tiles_n, num_tiles, nkb);
+    gemm_epilogue<BN>(sm, tmem_base, args, &tmC, &tmR, tiles_m, tiles_n, num_tiles, nkb);
   }
 
   tc_fence_before();
@@ -333,8 +379,8 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
 }
 
 template <int BN>
-cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& a, int num_sms,
-                      cudaStream_t st) {
+cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
+                      const CUtensorMap& tmR, const GemmArgs& a, int num_sms, cudaStream_t st) {
   using Cfg = GemmCfg<BN>;
   cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)Cfg::SMEM);
@@ -348,7 +394,7 @@ cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const Gemm
   }
   const int tiles = ((a.M + 127) / 128) * ((a.N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  fp8_gemm_kernel<BN><<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(tmA, tmB, a);
+  fp8_gemm_kernel<BN><<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(tmA, tmB, tmC, tmR, a);
   return cudaGetLastError();
 }
 
@@ -358,14 +404,19 @@ cudaError_t launch_fp8_gemm(const uint8_t* A, const float* sA, int ldsA, const u
                             const __nv_bfloat16* bias, const __nv_bfloat16* residual, __nv_bfloat16* C,
                             int M, int N, int K, int block_n, int num_sms, cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmC, tmR;
   const int bn = block_n == 256 ? 256 : 128;
   cudaError_t e = encode_tma_2d_u8(&tmA, A, K, M, 128, 128);
   if (e != cudaSuccess) return e;
   e = encode_tma_2d_u8(&tmB, W, K, N, 128, bn);
   if (e != cudaSuccess) return e;
+  e = encode_tma_2d_bf16(&tmC, C, N, M, 64, 32);
+  if (e != cudaSuccess) return e;
+  e = encode_tma_2d_bf16(&tmR, residual ? residual : C, N, M, 64, 32);
+  if (e != cudaSuccess) return e;
   GemmArgs a{sA, ldsA, sW, bias, residual, C, M, N, K};
-  return bn == 256 ? launch_bn<256>(tmA, tmB, a, num_sms, st) : launch_bn<128>(tmA, tmB, a, num_sms, st);
+  return bn == 256 ? launch_bn<256>(tmA, tmB, tmC, tmR, a, num_sms, st)
+                   : launch_bn<128>(tmA, tmB, tmC, tmR, a, num_sms, st);
 }
 
 }  // namespace vitq

@@ -20,6 +20,10 @@ struct GridList {
 // 2D uint8 matrix [rows, cols] (row pitch = cols bytes), box {box_cols, box_rows}, 128B swizzle.
 cudaError_t encode_tma_2d_u8(CUtensorMap* tm, const void* base, int cols, int rows, int box_cols,
                              int box_rows);
+// 2D bf16 matrix [rows, cols] (row pitch = cols * 2 bytes), box {box_cols, box_rows}, 128B swizzle
+// (box_cols = 64).
+cudaError_t encode_tma_2d_bf16(CUtensorMap* tm, const void* base, int cols, int rows, int box_cols,
+                               int box_rows);
 // Packed qkv [n, 3, 16, 72] bf16 viewed as 3D (d = 72, slot = 48, token = n); box {box_d, 1, 128}.
 // lo = true: 128B swizzle (box_d = 64); lo = false: 32B swizzle (box_d = 16).
 cudaError_t encode_tma_qkv(CUtensorMap* tm, const void* qkv, int n_tokens, int box_d, bool lo);
