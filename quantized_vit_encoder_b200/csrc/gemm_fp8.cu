@@ -45,7 +45,7 @@ struct GemmCfg {
   static constexpr bool SPLIT_REGS = BN == 256;
   static constexpr int MIN_LAUNCH_REGS = 168;   // 384 x 168 >= 128 x 56 + 256 x 224 (BN = 256)
   static constexpr int OUT_WARP_BYTES = 2 * 4096;   // two 64-column SW128 boxes of 32 rows
-  static constexpr int OUT_BYTES = EPI_WARPS * OUT_WARP_BYTES;
+  static constexpr int OUT_BYTES = EPI_WARPS * (OUT_WARP_BYTES + 256);   // + the warp's 128 bias values
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF + EPI_WARPS) * 8 + 16;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + OUT_BYTES + 1024 + BAR_BYTES;
 };
@@ -71,6 +71,9 @@ struct GemmSmem {
   }
   __device__ uint8_t* out(int w) const {
     return base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + (size_t)w * Cfg::OUT_WARP_BYTES;
+  }
+  __device__ uint8_t* bias(int w) const {
+    return base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + (size_t)Cfg::EPI_WARPS * Cfg::OUT_WARP_BYTES + w * 256;
   }
   __device__ uint64_t* bars() const {
     return reinterpret_cast<uint64_t*>(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES);
@@ -202,17 +205,21 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
     const int y0 = m0 + quad * 32;                   // first row of this warp's staging tile
     const bool row_ok = row < g.M;
     const bool col_ok = col0 < g.N;
-    // the staging tile is free once the previous tile's stores have read it;
-    // then the residual tile (if any) is fetched into it during the K loop
-    if (lane == 0) {
-      bulk_wait_read_all();
-      if (has_res) {
+    // this warp's 128 bias values (lane l: columns 4l..4l+3), loaded now and
+    // parked in shared memory after the K loop
+    uint2 bias_l = make_uint2(0u, 0u);
+    if (g.bias && col0 + 4 * lane < g.N) bias_l = __ldg(reinterpret_cast<const uint2*>(g.bias + col0 + 4 * lane));
+    // the residual tile is requested at the start of the tile, once the previous
+    // tile's stores have read the staging tile
+    if (has_res) {
+      if (lane == 0) {
+        bulk_wait_read_all();
         mbar_arrive_expect_tx(sm.res_full(ew), Cfg::OUT_WARP_BYTES);
         tma_load_2d(stg_u32, tmR, col0, y0, sm.res_full(ew));
         tma_load_2d(stg_u32 + 4096, tmR, col0 + 64, y0, sm.res_full(ew));
       }
+      __syncwarp();
     }
-    __syncwarp();
     const float* sa_ptr = g.sA + row;
     const float* sw_ptr = g.sW + (size_t)(col0 >> 7) * nkb;
     uint64_t acc[64];
@@ -255,10 +262,17 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
       if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(6, cnt);  // epilogue: partial consumed
       if (lane == 0) mbar_arrive(sm.tempty(buf));
     }
+    if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(7, it);  // epilogue: K loop done
+    uint8_t* bias_s = sm.bias(ew);
+    *reinterpret_cast<uint2*>(bias_s + lane * 8) = bias_l;
     if (has_res) {
       const bool ok = mbar_wait(sm.res_full(ew), it & 1u, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
+    } else {
+      if (lane == 0) bulk_wait_read_all();   // the previous tile's stores have read the staging tile
     }
+    __syncwarp();
+    if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(9, it);  // epilogue: staging free
     // bias + residual, bf16, into the staging tile (row = lane, 16-byte chunk c of
     // box h at position c ^ (lane & 7))
 #pragma unroll
@@ -266,7 +280,6 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const int c8 = h * 8 + c;
-        const int col = col0 + c8 * 8;
         float v[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -274,8 +287,8 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
           v[2 * i] = f.x;
           v[2 * i + 1] = f.y;
         }
-        if (g.bias && col < g.N) {
-          const uint4 bu = __ldg(reinterpret_cast<const uint4*>(g.bias + col));
+        if (g.bias) {
+          const uint4 bu = *reinterpret_cast<const uint4*>(bias_s + c8 * 16);
           const uint32_t bw[4] = {bu.x, bu.y, bu.z, bu.w};
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -305,6 +318,7 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
     }
     fence_proxy_async_smem();
     __syncwarp();
+    if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(8, it);  // epilogue: staging written
     if (lane == 0) {
       // TMA clips rows >= M and columns >= N; boxes wholly outside are skipped
       if (y0 < g.M) {
