@@ -194,6 +194,12 @@ TowerWs carve_tower_head(Carver& c, int n, int n_images) {
     if (!(cond)) return (code); \
   } while (0)
 
+// CTA pairs (cta_group::2 MMA) for the GEMMs; VITQ_GEMM_PAIR=0 selects one CTA per tile.
+bool pick_pair() {
+  if (const char* env = std::getenv("VITQ_GEMM_PAIR")) return std::atoi(env) != 0;
+  return false;
+}
+
 int gemm_checked(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W, const float* sW,
                  const void* bias, const void* residual, void* C, int M, int N, int K, int num_sms,
                  cudaStream_t st) {
@@ -203,7 +209,7 @@ int gemm_checked(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W, 
               launch_fp8_gemm(A, sA, ldsA, W, sW, reinterpret_cast<const __nv_bfloat16*>(bias),
                            reinterpret_cast<const __nv_bfloat16*>(residual),
                            reinterpret_cast<__nv_bfloat16*>(C), M, N, K, pick_block_n(M, N, num_sms),
-                           num_sms, st));
+                           pick_pair(), num_sms, st));
   return VITQ_OK;
 }
 

@@ -7,7 +7,12 @@
 // weight scales), with the bias adds and the residual fused into the GEMM.
 //
 // Design (B200):
-//   * persistent CTAs, one per SM, walking 128 x BN output tiles;
+//   * persistent CTAs, one per SM, walking 128 x BN output tiles; or, with
+//     kPair, clusters of two CTAs walking 256 x BN tiles: each CTA loads its
+//     128 rows of A and half of the BN rows of W, and the leader issues
+//     cta_group::2 MMAs that read both CTAs' shared memory and write both
+//     CTAs' TMEM, so each SM fetches 16 + BN/2 x 128 bytes per K block instead
+//     of 16 + BN x 128 (the K loop is bound by that operand supply);
 //   * warp 0: TMA producer (A and W tiles of 128 K-columns into a multi-stage
 //     128B-swizzled shared-memory ring, zero fill past K / M / N);
 //   * warp 1: MMA issuer, 4 x tcgen05.mma kind::f8f6f4 (K = 32 each) per K
@@ -31,15 +36,18 @@ namespace {
 // BN = 128: 6 warps (TMA, MMA, 4 epilogue warps).  BN = 256: 12 warps
 // (warpgroup 0 = TMA, MMA and two idle warps, which give registers away with
 // setmaxnreg; warpgroups 1-2 = 8 epilogue warps, one per 128 columns x 32 rows).
-template <int BN>
+template <int BN, bool kPair = false>
 struct GemmCfg {
-  static constexpr int BM = 128, BK = 128;
-  static constexpr int STAGES = BN == 256 ? 3 : 5;
+  static constexpr int BM = 128, BK = 128;            // rows of A per CTA, K per stage
+  static constexpr int TILE_M = kPair ? 256 : 128;    // rows per output tile
+  static constexpr int B_ROWS = kPair ? BN / 2 : BN;  // rows of W loaded per CTA
+  static constexpr int STAGES = kPair ? (BN == 256 ? 4 : 7) : (BN == 256 ? 3 : 5);
   static constexpr int A_BYTES = BM * BK;
-  static constexpr int B_BYTES = BN * BK;
+  static constexpr int B_BYTES = B_ROWS * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NBUF = 512 / BN;
   static constexpr int EPI_WARPS = BN / 32;
+  static constexpr int TEMPTY_COUNT = EPI_WARPS * (kPair ? 2 : 1);   // both CTAs' epilogues free a buffer
   static constexpr int EPI_WARP0 = BN == 256 ? 4 : 2;
   static constexpr int THREADS = BN == 256 ? 384 : 192;
   static constexpr bool SPLIT_REGS = BN == 256;
@@ -61,9 +69,9 @@ struct GemmArgs {
   int M, N, K;
 };
 
-template <int BN>
+template <int BN, bool kPair>
 struct GemmSmem {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, kPair>;
   uint8_t* base;
   __device__ uint32_t a(int s) const { return smem_u32(base + (size_t)s * Cfg::STAGE_BYTES); }
   __device__ uint32_t b(int s) const {
@@ -105,23 +113,32 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
   n = VITQ_GEMM_DIAG ? (q + m) % tiles_n : q;
 }
 
-template <int BN>
-__device__ void gemm_producer(const GemmSmem<BN>& sm, const CUtensorMap* tmA, const CUtensorMap* tmB,
-                              int tiles_m, int tiles_n, int num_tiles, int nkb) {
-  using Cfg = GemmCfg<BN>;
+// Tiles of this CTA (or CTA pair): t0, t0 + dt, ...
+template <int BN, bool kPair>
+__device__ void gemm_producer(const GemmSmem<BN, kPair>& sm, const CUtensorMap* tmA, const CUtensorMap* tmB,
+                              int tiles_m, int tiles_n, int num_tiles, int nkb, int t0, int dt, int rank) {
+  using Cfg = GemmCfg<BN, kPair>;
   int stage = 0;
   uint32_t phase = 0;
-  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+  for (int tile = t0; tile < num_tiles; tile += dt) {
     int mt, nt;
     tile_coords(tile, tiles_m, tiles_n, mt, nt);
-    const int m0 = mt * Cfg::BM;
-    const int n0 = nt * BN;
+    const int m0 = mt * Cfg::TILE_M + rank * Cfg::BM;
+    const int n0 = nt * BN + rank * Cfg::B_ROWS;
     for (int kb = 0; kb < nkb; ++kb) {
       if (!mbar_wait(sm.empty(stage), phase ^ 1u, sm.abort_flag())) return;
-      VITQ_TRACE_EV(1, (tile - (int)blockIdx.x) / (int)gridDim.x * nkb + kb);  // producer: stage free, issuing loads
-      mbar_arrive_expect_tx(sm.full(stage), Cfg::STAGE_BYTES);
-      tma_load_2d(sm.a(stage), tmA, kb * Cfg::BK, m0, sm.full(stage));
-      tma_load_2d(sm.b(stage), tmB, kb * Cfg::BK, n0, sm.full(stage));
+      VITQ_TRACE_EV(1, (tile - t0) / dt * nkb + kb);  // producer: stage free, issuing loads
+      if (kPair) {
+        // both CTAs' copies count on the leader's full barrier, which expects them all
+        const uint32_t full0 = mapa_shared(sm.full(stage), 0);
+        if (rank == 0) mbar_arrive_expect_tx(sm.full(stage), 2 * Cfg::STAGE_BYTES);
+        tma_load_2d_pair(sm.a(stage), tmA, kb * Cfg::BK, m0, full0);
+        tma_load_2d_pair(sm.b(stage), tmB, kb * Cfg::BK, n0, full0);
+      } else {
+        mbar_arrive_expect_tx(sm.full(stage), Cfg::STAGE_BYTES);
+        tma_load_2d(sm.a(stage), tmA, kb * Cfg::BK, m0, sm.full(stage));
+        tma_load_2d(sm.b(stage), tmB, kb * Cfg::BK, n0, sm.full(stage));
+      }
       if (++stage == Cfg::STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -130,14 +147,15 @@ __device__ void gemm_producer(const GemmSmem<BN>& sm, const CUtensorMap* tmA, co
   }
 }
 
-template <int BN>
-__device__ void gemm_mma(const GemmSmem<BN>& sm, uint32_t tmem_base, int num_tiles, int nkb) {
-  using Cfg = GemmCfg<BN>;
-  constexpr uint32_t idesc = make_idesc(0, 0, 0, 0, 128, BN);
+template <int BN, bool kPair>
+__device__ void gemm_mma(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base, int num_tiles, int nkb, int t0,
+                         int dt) {
+  using Cfg = GemmCfg<BN, kPair>;
+  constexpr uint32_t idesc = make_idesc(0, 0, 0, 0, Cfg::TILE_M, BN);
   int stage = 0;
   uint32_t phase = 0;
   uint32_t cnt = 0;
-  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+  for (int tile = t0; tile < num_tiles; tile += dt) {
     for (int kb = 0; kb < nkb; ++kb, ++cnt) {
       const uint32_t buf = cnt % Cfg::NBUF;
       const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
@@ -152,10 +170,18 @@ __device__ void gemm_mma(const GemmSmem<BN>& sm, uint32_t tmem_base, int num_til
       for (int k = 0; k < 4; ++k) {
         const uint64_t ad = make_smem_desc(a0 + 32 * k, 16, 1024, kSwizzle128B);
         const uint64_t bd = make_smem_desc(b0 + 32 * k, 16, 1024, kSwizzle128B);
-        mma_f8_ss(tmem_base + buf * BN, ad, bd, idesc, k > 0 ? 1u : 0u);
+        if (kPair)
+          mma_f8_ss_pair(tmem_base + buf * BN, ad, bd, idesc, k > 0 ? 1u : 0u);
+        else
+          mma_f8_ss(tmem_base + buf * BN, ad, bd, idesc, k > 0 ? 1u : 0u);
       }
-      tc_commit(sm.empty(stage));
-      tc_commit(sm.tfull(buf));
+      if (kPair) {   // release the stage in both CTAs; both epilogues may read their TMEM
+        tc_commit_pair(sm.empty(stage), 0x3);
+        tc_commit_pair(sm.tfull(buf), 0x3);
+      } else {
+        tc_commit(sm.empty(stage));
+        tc_commit(sm.tfull(buf));
+      }
       if (++stage == Cfg::STAGES) {
         stage = 0;
         phase ^= 1u;
@@ -181,11 +207,11 @@ __device__ __forceinline__ uint64_t fma2(uint64_t p, uint64_t s, uint64_t acc) {
   return d;
 }
 
-template <int BN>
-__device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const GemmArgs& g,
+template <int BN, bool kPair>
+__device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base, const GemmArgs& g,
                               const CUtensorMap* tmC, const CUtensorMap* tmR, int tiles_m, int tiles_n,
-                              int num_tiles, int nkb) {
-  using Cfg = GemmCfg<BN>;
+                              int num_tiles, int nkb, int t0, int dt, int rank) {
+  using Cfg = GemmCfg<BN, kPair>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;                         // TMEM lane quadrant this warp may access
   const int ew = warp - Cfg::EPI_WARP0;              // epilogue warp index
@@ -194,11 +220,13 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
   uint8_t* stg = sm.out(ew);                         // staging: [2 boxes][32 rows][128 B], SW128
   const uint32_t stg_u32 = smem_u32(stg);
   const bool has_res = g.residual != nullptr;
+  // the leader's tempty barriers count both CTAs' epilogue warps
+  const uint32_t tempty0 = kPair ? mapa_shared(sm.tempty(0), 0) : sm.tempty(0);
   uint32_t cnt = 0, it = 0;
-  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+  for (int tile = t0; tile < num_tiles; tile += dt, ++it) {
     int mt, nt;
     tile_coords(tile, tiles_m, tiles_n, mt, nt);
-    const int m0 = mt * Cfg::BM;
+    const int m0 = mt * Cfg::TILE_M + rank * Cfg::BM;
     const int n0 = nt * BN;
     const int row = m0 + r_in;
     const int col0 = n0 + cg * 128;
@@ -260,7 +288,12 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
       tc_fence_before();
       __syncwarp();
       if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(6, cnt);  // epilogue: partial consumed
-      if (lane == 0) mbar_arrive(sm.tempty(buf));
+      if (lane == 0) {
+        if (kPair)
+          mbar_arrive_cluster(tempty0 + buf * 8);
+        else
+          mbar_arrive(sm.tempty(buf));
+      }
     }
     if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(7, it);  // epilogue: K loop done
     uint8_t* bias_s = sm.bias(ew);
@@ -331,20 +364,24 @@ __device__ void gemm_epilogue(const GemmSmem<BN>& sm, uint32_t tmem_base, const 
   if (lane == 0) bulk_wait_all();
 }
 
-template <int BN>
-__global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
+template <int BN, bool kPair>
+__global__ void __launch_bounds__(GemmCfg<BN, kPair>::THREADS, 1)
     fp8_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmC, const __grid_constant__ CUtensorMap tmR,
                     const GemmArgs args) {
-  using Cfg = GemmCfg<BN>;
+  using Cfg = GemmCfg<BN, kPair>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  GemmSmem<BN> sm;
+  GemmSmem<BN, kPair> sm;
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkb = (args.K + Cfg::BK - 1) / Cfg::BK;
-  const int tiles_m = (args.M + Cfg::BM - 1) / Cfg::BM;
+  const int tiles_m = (args.M + Cfg::TILE_M - 1) / Cfg::TILE_M;
   const int tiles_n = (args.N + BN - 1) / BN;
   const int num_tiles = tiles_m * tiles_n;
+  // a CTA pair walks the tiles as one unit
+  const int rank = kPair ? (int)cluster_ctarank() : 0;
+  const int t0 = kPair ? (int)blockIdx.x / 2 : (int)blockIdx.x;
+  const int dt = kPair ? (int)gridDim.x / 2 : (int)gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -353,15 +390,21 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     }
     for (int b = 0; b < Cfg::NBUF; ++b) {
       mbar_init(sm.tfull(b), 1);
-      mbar_init(sm.tempty(b), Cfg::EPI_WARPS);
+      mbar_init(sm.tempty(b), Cfg::TEMPTY_COUNT);
     }
     for (int w = 0; w < Cfg::EPI_WARPS; ++w) mbar_init(sm.res_full(w), 1);
     *sm.abort_flag() = 0;
     fence_barrier_init();
   }
+  if (kPair) cluster_sync_all();   // the peer's barriers exist before anything signals them
   if (warp == 1) {
-    tmem_alloc(smem_u32(sm.tmem_holder()), 512);
-    tmem_relinquish();
+    if (kPair) {
+      tmem_alloc_pair(smem_u32(sm.tmem_holder()), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(sm.tmem_holder()), 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -373,64 +416,90 @@ __global__ void __launch_bounds__(GemmCfg<BN>::THREADS, 1)
     if (warp == 0 && lane == 0) {
       prefetch_tensormap(&tmA);
       prefetch_tensormap(&tmB);
-      gemm_producer<BN>(sm, &tmA, &tmB, tiles_m, tiles_n, num_tiles, nkb);
-    } else if (warp == 1 && lane == 0) {
-      gemm_mma<BN>(sm, tmem_base, num_tiles, nkb);
+      gemm_producer<BN, kPair>(sm, &tmA, &tmB, tiles_m, tiles_n, num_tiles, nkb, t0, dt, rank);
+    } else if (warp == 1 && lane == 0 && rank == 0) {
+      gemm_mma<BN, kPair>(sm, tmem_base, num_tiles, nkb, t0, dt);
     }
   } else {
     if (Cfg::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
-    gemm_epilogue<BN>(sm, tmem_base, args, &tmC, &tmR, tiles_m, tiles_n, num_tiles, nkb);
+    gemm_epilogue<BN, kPair>(sm, tmem_base, args, &tmC, &tmR, tiles_m, tiles_n, num_tiles, nkb, t0, dt, rank);
   }
 
   tc_fence_before();
   __syncthreads();
   if (*sm.abort_flag()) settle_pause(50000);
+  // neither CTA of a pair leaves while the leader's MMAs may still use the
+  // peer's shared memory and TMEM (all of them completed before the last
+  // partial was consumed by both epilogues)
+  if (kPair) cluster_sync_all();
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 512);
+    if (kPair)
+      tmem_dealloc_pair(tmem_base, 512);
+    else
+      tmem_dealloc(tmem_base, 512);
   }
 }
 
-template <int BN>
+template <int BN, bool kPair>
 cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUtensorMap& tmC,
                       const CUtensorMap& tmR, const GemmArgs& a, int num_sms, cudaStream_t st) {
-  using Cfg = GemmCfg<BN>;
-  cudaError_t e = cudaFuncSetAttribute(fp8_gemm_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)Cfg::SMEM);
+  using Cfg = GemmCfg<BN, kPair>;
+  auto kern = fp8_gemm_kernel<BN, kPair>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg::SMEM);
   if (e != cudaSuccess) return e;
   if (Cfg::SPLIT_REGS) {
     // setmaxnreg.inc only draws on the registers the CTA was launched with.
     cudaFuncAttributes fa;
-    e = cudaFuncGetAttributes(&fa, fp8_gemm_kernel<BN>);
+    e = cudaFuncGetAttributes(&fa, kern);
     if (e != cudaSuccess) return e;
     if (fa.numRegs < Cfg::MIN_LAUNCH_REGS) return cudaErrorInvalidConfiguration;
   }
-  const int tiles = ((a.M + 127) / 128) * ((a.N + BN - 1) / BN);
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  fp8_gemm_kernel<BN><<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(tmA, tmB, tmC, tmR, a);
-  return cudaGetLastError();
+  const int tiles = ((a.M + Cfg::TILE_M - 1) / Cfg::TILE_M) * ((a.N + BN - 1) / BN);
+  if (!kPair) {
+    const int grid = tiles < num_sms ? tiles : num_sms;
+    kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(tmA, tmB, tmC, tmR, a);
+    return cudaGetLastError();
+  }
+  const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = Cfg::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmC, tmR, a);
 }
 
 }  // namespace
 
 cudaError_t launch_fp8_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W, const float* sW,
                             const __nv_bfloat16* bias, const __nv_bfloat16* residual, __nv_bfloat16* C,
-                            int M, int N, int K, int block_n, int num_sms, cudaStream_t st) {
+                            int M, int N, int K, int block_n, bool pair, int num_sms, cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
   CUtensorMap tmA, tmB, tmC, tmR;
   const int bn = block_n == 256 ? 256 : 128;
   cudaError_t e = encode_tma_2d_u8(&tmA, A, K, M, 128, 128);
   if (e != cudaSuccess) return e;
-  e = encode_tma_2d_u8(&tmB, W, K, N, 128, bn);
+  e = encode_tma_2d_u8(&tmB, W, K, N, 128, pair ? bn / 2 : bn);
   if (e != cudaSuccess) return e;
   e = encode_tma_2d_bf16(&tmC, C, N, M, 64, 32);
   if (e != cudaSuccess) return e;
   e = encode_tma_2d_bf16(&tmR, residual ? residual : C, N, M, 64, 32);
   if (e != cudaSuccess) return e;
   GemmArgs a{sA, ldsA, sW, bias, residual, C, M, N, K};
-  return bn == 256 ? launch_bn<256>(tmA, tmB, tmC, tmR, a, num_sms, st)
-                   : launch_bn<128>(tmA, tmB, tmC, tmR, a, num_sms, st);
+  if (pair)
+    return bn == 256 ? launch_bn<256, true>(tmA, tmB, tmC, tmR, a, num_sms, st)
+                     : launch_bn<128, true>(tmA, tmB, tmC, tmR, a, num_sms, st);
+  return bn == 256 ? launch_bn<256, false>(tmA, tmB, tmC, tmR, a, num_sms, st)
+                   : launch_bn<128, false>(tmA, tmB, tmC, tmR, a, num_sms, st);
 }
 
 }  // namespace vitq

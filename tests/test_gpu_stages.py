@@ -174,11 +174,14 @@ GEMM_SHAPES = [
 ]
 
 
+@pytest.mark.parametrize("pair", [0, 1], ids=["cta", "pair"])
 @pytest.mark.parametrize("bn", [128, 256])
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
-def test_fp8_gemm_matches_oracle(lib, monkeypatch, bn, M, N, K):
+def test_fp8_gemm_matches_oracle(lib, monkeypatch, pair, bn, M, N, K):
+    """One CTA per tile and CTA pairs (cta_group::2 MMA over 256-row tiles)."""
     from quantized_vit_encoder_b200 import vitq
     monkeypatch.setenv("VITQ_GEMM_BN", str(bn))
+    monkeypatch.setenv("VITQ_GEMM_PAIR", str(pair))
     a = bf16((M, K), 50 + M, 1.0)
     w = bf16((N, K), 51 + N, 0.02)
     bias = bf16((N,), 52, 0.01)
@@ -194,7 +197,7 @@ def test_fp8_gemm_matches_oracle(lib, monkeypatch, bn, M, N, K):
                               torch.from_numpy(qw).to(dev), torch.from_numpy(sw).to(dev),
                               bias.to(dev), res.to(dev))
     got = f64(out)
-    assert_close(got, ref, what=f"gemm {M}x{N}x{K} bn{bn}")
+    assert_close(got, ref, what=f"gemm {M}x{N}x{K} bn{bn} pair{pair}")
     # the promotion is fp32 against an fp64 oracle: nearly every bf16 output is identical
     assert np.mean(got == ref) > 0.97
 
