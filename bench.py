@@ -220,6 +220,48 @@ def _source_sha(rel: str) -> str | None:
     return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
 
 
+def graph_study(tower, ws, dev, steps: int = 5) -> dict:
+    """Tower step through the C ABI launched one kernel at a time vs replayed as one
+    CUDA graph (captured once, the library's launches unchanged), at 256, 972 and
+    6256 patches.  Device time per step from CUDA events on the launching stream."""
+    from quantized_vit_encoder_b200 import vitq
+    out = {}
+    for name, grids in (("16x16", [(16, 16)]), ("54x18", [(54, 18)]), ("46x136", [(46, 136)])):
+        n = sum(h * w for h, w in grids)
+        x0 = wl.random_bf16((n, wl.HIDDEN), 77, 1.0).to(dev)
+        x = torch.empty_like(x0)
+        taps = [torch.empty((n // 4, wl.OUT_HIDDEN), dtype=torch.bfloat16, device=dev) for _ in range(4)]
+
+        def step():
+            x.copy_(x0)
+            vitq.tower_forward_(tower, x, grids, ws, taps)
+
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            for _ in range(2):
+                step()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step()
+        st = torch.cuda.current_stream(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        res = {"patches": n}
+        for mode, fn in (("eager_ms", step), ("graph_ms", g.replay)):
+            fn()
+            torch.cuda.synchronize(dev)
+            e0.record(st)
+            for _ in range(steps):
+                fn()
+            e1.record(st)
+            torch.cuda.synchronize(dev)
+            res[mode] = e0.elapsed_time(e1) / steps
+        del g
+        out[name] = res
+    return out
+
+
 def run_gpu(args, rank: int, world: int, local_rank: int):
     from quantized_vit_encoder_b200 import vitq
     torch.cuda.set_device(local_rank)
@@ -315,6 +357,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     barrier()
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
 
+    graphs = graph_study(tower, ws, dev) if world == 1 else None
+
     if rank != 0:
         return
     peaks = load_peaks()
@@ -341,6 +385,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "kernel_shapes": {k: {"launches": v["launches"] // 2, "us_per_launch": 1e3 * v["ms"] / v["launches"]}
                           for k, v in sorted(shapes.items(), key=lambda kv: -kv[1]["ms"])},
         "gpu_launches": int(launches),
+        "graph_study": graphs,
         "clocks": clk.summary(),
         "e2e": {"value": world * fl["tower"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},

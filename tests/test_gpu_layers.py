@@ -135,6 +135,44 @@ def test_full_tower_deterministic_and_finite(lib):
         assert torch.equal(a, b)
 
 
+def test_tower_graph_replay_equals_stream_launches(lib):
+    """The tower captured once in a CUDA graph and replayed gives bitwise the taps of
+    the same call launched kernel by kernel (the entry points allocate nothing and
+    synchronise nothing after their first call, so they can be captured)."""
+    from quantized_vit_encoder_b200 import vitq
+    W = wl.Workload("tower_graph", ((16, 16), (8, 12)), wl.N_BLOCKS, True, scales=(1.0, 2.0), seed_base=5100)
+    x0 = wl.make_input(W).cuda()
+    tower = _device_tower(W)
+    ws = vitq.workspace(vitq.tower_workspace_bytes(W.n_tokens, len(W.grids)))
+    x = torch.empty_like(x0)
+    taps = [torch.empty((W.n_tokens // 4, wl.OUT_HIDDEN), dtype=torch.bfloat16, device="cuda") for _ in range(4)]
+
+    def step():
+        x.copy_(x0)
+        vitq.tower_forward_(tower, x, list(W.grids), ws, taps)
+
+    step()
+    eager = [t.clone() for t in taps]
+    for t in taps:
+        t.zero_()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for t in taps:
+        t.zero_()
+    g.replay()
+    g.replay()
+    torch.cuda.synchronize()
+    assert vitq.device_error() == 0
+    for a, b in zip(taps, eager):
+        assert torch.equal(a, b)
+
+
 def test_packed_tower_equals_per_image_towers(lib):
     """Block-diagonal attention and row-wise stages: each image of the packed 4-image batch
     (9164 patches) gives bitwise the same taps as that image run alone."""
