@@ -122,6 +122,16 @@ int vit_gelu_quant(const void* f, int M, int K, int ldf, uint8_t* q, float* s, i
 int fp8_block_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W, const float* sW,
                    const void* bias, const void* residual, void* C, int M, int N, int K, void* stream);
 
+/* bf16 GEMM with fused bias and residual, fp32 accumulation over all of K
+ * ([FRT] s4: the patch embedding, the first three blocks and the mergers stay
+ * bf16; [VE] dense_gemm_bf16 / vision_gemm_bias):
+ *   C[m,n] = bf16( sum_k A[m,k] W[n,k] + bias[n] + residual[m,n] )
+ * A: bf16 [M, K]; W: bf16 [N, K]; bias bf16 [N] or NULL; residual bf16 [M, N]
+ * or NULL (may equal C); C bf16 [M, N].  K % 8 == 0, N % 8 == 0; all pointers
+ * 16-byte aligned.  The K tail (K % 64) is zero-filled in shared memory. */
+int bf16_gemm(const void* A, const void* W, const void* bias, const void* residual, void* C, int M, int N, int K,
+              void* stream);
+
 /* 2D rotary table ([FRT] s3 "2D rotate_half RoPE"; [VE] rope_inv_freq, head_dim/4
  * entries).  pos_hw: int32 [n][2] (row, col) per token.  Output cos_sin fp32
  * [n][72]: cos of the 36 angles then their sines; angle j = row * f_j for

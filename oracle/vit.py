@@ -135,6 +135,22 @@ def fp8_block_gemm(qa, sa, qw, sw, bias=None, residual=None) -> np.ndarray:
     return bf16_round(acc)
 
 
+def bf16_gemm(a, w, bias=None, residual=None) -> np.ndarray:
+    """C[m, n] = bf16( sum_k a[m, k] w[n, k] + bias[n] + residual[m, n] ) for bf16 a, w.
+
+    The bf16 linears of [FRT s4] (patch embedding, first three blocks,
+    mergers) and [VE] dense_gemm_bf16 + vision_add_bias: the plain matrix
+    product of the bf16 values, taken in fp64 (a library matmul as one step),
+    then one bf16 rounding after the bias and residual adds.
+    """
+    acc = np.asarray(a, np.float64) @ np.asarray(w, np.float64).T
+    if bias is not None:
+        acc = acc + np.asarray(bias, np.float64)[None, :]
+    if residual is not None:
+        acc = acc + np.asarray(residual, np.float64)
+    return bf16_round(acc)
+
+
 # --------------------------------------------------------------------------
 # LayerNorm and GELU  [FRT s3: "LayerNorm", "GELU(tanh)"; VE norm1_w/b]
 # --------------------------------------------------------------------------

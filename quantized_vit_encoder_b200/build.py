@@ -9,7 +9,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libvitq.so")
-SOURCES = ["vitq_all.cu", "elementwise.cu", "gemm_fp8.cu", "attention.cu", "api.cu", "merger_static.cu",
+SOURCES = ["vitq_all.cu", "elementwise.cu", "gemm_fp8.cu", "gemm_bf16.cu", "attention.cu", "api.cu", "merger_static.cu",
            "ptx.cuh", "internal.h"]
 
 

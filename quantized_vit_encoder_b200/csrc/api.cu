@@ -213,6 +213,16 @@ int gemm_checked(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W, 
   return VITQ_OK;
 }
 
+int bf16_gemm_checked(const __nv_bfloat16* A, const __nv_bfloat16* W, const __nv_bfloat16* bias,
+                      const __nv_bfloat16* residual, __nv_bfloat16* C, int M, int N, int K, int num_sms,
+                      cudaStream_t st) {
+  const double mn = (double)M * N;
+  VITQ_LAUNCH("bf16_gemm", st, 2.0 * mn * K,
+              2.0 * ((double)M * K + (double)N * K) + mn * 2 * (residual ? 2 : 1),
+              launch_bf16_gemm(A, W, bias, residual, C, M, N, K, pick_block_n(M, N, num_sms), num_sms, st));
+  return VITQ_OK;
+}
+
 bool block_weights_ok(const vitq_block_weights* w) {
   return w && w->norm1_w && w->norm1_b && w->qkv_q && w->qkv_s && w->qkv_b && w->proj_q && w->proj_s &&
          w->proj_b && w->norm2_w && w->norm2_b && w->fc1_q && w->fc1_s && w->fc1_b && w->fc2_q &&
@@ -386,6 +396,20 @@ int fp8_block_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W
   int r = current_device_ok(&sms);
   if (r) return r;
   return gemm_checked(A, sA, ldsA, W, sW, bias, residual, C, M, N, K, sms, S(stream));
+}
+
+int bf16_gemm(const void* A, const void* W, const void* bias, const void* residual, void* C, int M, int N, int K,
+              void* stream) {
+  VITQ_CHECK(A && W && C, VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(M >= 0 && N > 0 && K > 0, VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(K % 8 == 0 && N % 8 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(al16(A) && al16(W) && al16(C) && (!bias || al16(bias)) && (!residual || al16(residual)),
+             VITQ_ERR_ALIGN);
+  int sms = 0;
+  int r = current_device_ok(&sms);
+  if (r) return r;
+  return bf16_gemm_checked((const __nv_bfloat16*)A, (const __nv_bfloat16*)W, (const __nv_bfloat16*)bias,
+                           (const __nv_bfloat16*)residual, (__nv_bfloat16*)C, M, N, K, sms, S(stream));
 }
 
 int vit_rope_table(const int32_t* pos_hw, int n_tokens, float theta, float* cos_sin, void* stream) {

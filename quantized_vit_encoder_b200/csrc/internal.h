@@ -46,6 +46,10 @@ cudaError_t launch_positions(const GridList& g, int n_total, int32_t* pos, int32
 cudaError_t launch_fp8_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W, const float* sW,
                             const __nv_bfloat16* bias, const __nv_bfloat16* residual, __nv_bfloat16* C,
                             int M, int N, int K, int block_n, bool pair, int num_sms, cudaStream_t st);
+// bf16 GEMM: C = A W^T + bias + residual (fp32 accumulation), A [M, K], W [N, K].
+cudaError_t launch_bf16_gemm(const __nv_bfloat16* A, const __nv_bfloat16* W, const __nv_bfloat16* bias,
+                             const __nv_bfloat16* residual, __nv_bfloat16* C, int M, int N, int K, int block_n,
+                             int num_sms, cudaStream_t st);
 cudaError_t launch_attention(const __nv_bfloat16* qkv, int n_tokens, const int32_t* cu, int n_seqs,
                              int max_seqlen, float scale, bool v_f16, __nv_bfloat16* out, cudaStream_t st);
 

@@ -45,6 +45,7 @@ _SIGS = {
     "vit_ln_quant": [_vp, _i, _i, _i, _vp, _vp, _f, _vp, _vp, _i, _vp],
     "vit_gelu_quant": [_vp, _i, _i, _i, _vp, _vp, _i, _vp],
     "fp8_block_gemm": [_vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
+    "bf16_gemm": [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _vp],
     "vit_rope_table": [_vp, _i, _f, _vp, _vp],
     "vit_rope2d": [_vp, _i, _vp, _i, _vp],
     "vit_positions": [_vp, _i, _vp, _vp, _vp],
@@ -185,6 +186,16 @@ def fp8_block_gemm(qa, sa, qw, sw, bias=None, residual=None, out=None, stream=No
         out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.device)
     _check(load().fp8_block_gemm(_p(qa), _p(sa), sa.stride(0), _p(qw), _p(sw), _p(bias), _p(residual), _p(out),
                                  M, N, K, _stream(stream)), "fp8_block_gemm")
+    return out
+
+
+def bf16_gemm(a, w, bias=None, residual=None, out=None, stream=None):
+    """bf16 C [M, N] = a [M, K] w[N, K]^T (+ bias) (+ residual), fp32 accumulation."""
+    M, K = a.shape
+    N = w.shape[0]
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    _check(load().bf16_gemm(_p(a), _p(w), _p(bias), _p(residual), _p(out), M, N, K, _stream(stream)), "bf16_gemm")
     return out
 
 

@@ -202,6 +202,30 @@ def test_fp8_gemm_matches_oracle(lib, monkeypatch, pair, bn, M, N, K):
     assert np.mean(got == ref) > 0.97
 
 
+BF16_GEMM_SHAPES = [
+    (1, 128, 64), (128, 1152, 1536), (129, 3456, 1152), (300, 4304, 1152), (972, 1152, 4304),
+    (77, 136, 72), (6256, 1152, 1536),
+]
+
+
+@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("M,N,K", BF16_GEMM_SHAPES)
+def test_bf16_gemm_matches_oracle(lib, monkeypatch, bn, M, N, K):
+    """fp32 accumulation over all of K in TMEM against the fp64 oracle (ragged M, N and K tails)."""
+    from quantized_vit_encoder_b200 import vitq
+    monkeypatch.setenv("VITQ_GEMM_BN", str(bn))
+    a = bf16((M, K), 70 + M, 1.0)
+    w = bf16((N, K), 71 + N, 0.03)
+    bias = bf16((N,), 72, 0.01)
+    res = bf16((M, N), 73, 1.0)
+    ref = ov.bf16_gemm(f64(a), f64(w), f64(bias), f64(res))
+    got = f64(vitq.bf16_gemm(a.cuda(), w.cuda(), bias.cuda(), res.cuda()))
+    assert_close(got, ref, what=f"bf16 gemm {M}x{N}x{K} bn{bn}")
+    assert np.mean(got == ref) > 0.97
+    plain = f64(vitq.bf16_gemm(a.cuda(), w.cuda()))
+    assert_close(plain, ov.bf16_gemm(f64(a), f64(w)), what="bf16 gemm plain")
+
+
 def test_fp8_gemm_no_bias_no_residual(lib):
     from quantized_vit_encoder_b200 import vitq
     M, N, K = 200, 384, 640

@@ -233,6 +233,36 @@ def test_gemm_operand_orientation():
     assert np.array_equal(out, want)
 
 
+def test_bf16_gemm_matches_brute_force_loops():
+    """Every output is the bf16 rounding of an exactly summed dot product + bias + residual
+    (bf16 x bf16 products are exact in fp64; the sums are checked with Python's exact fsum)."""
+    g = np.random.default_rng(17)
+    M, N, K = 3, 10, 37
+    a = nm.bf16_round(g.standard_normal((M, K)))
+    w = nm.bf16_round(g.standard_normal((N, K)) * 0.1)
+    bias = nm.bf16_round(g.standard_normal(N) * 0.1)
+    res = nm.bf16_round(g.standard_normal((M, N)))
+    got = ov.bf16_gemm(a, w, bias, res)
+    for m in range(M):
+        for n in range(N):
+            exact = math.fsum([float(a[m, k]) * float(w[n, k]) for k in range(K)] + [float(bias[n]), float(res[m, n])])
+            assert abs(got[m, n] - exact) <= abs(exact) * 2.0 ** -8 + 1e-30
+
+
+def test_bf16_gemm_exact_integer_case_and_orientation():
+    g = np.random.default_rng(18)
+    A = g.integers(-3, 4, (4, 64)).astype(np.float64)
+    W = g.integers(-3, 4, (5, 64)).astype(np.float64)
+    assert np.array_equal(ov.bf16_gemm(A, W), nm.bf16_round(A @ W.T))   # exact integers, one rounding
+    a = np.zeros((4, 16))
+    w = np.zeros((6, 16))
+    a[2, 9], w[5, 9] = 3.0, 0.5
+    out = ov.bf16_gemm(a, w, bias=np.arange(6.0), residual=np.full((4, 6), 2.0))
+    want = np.tile(np.arange(6.0) + 2.0, (4, 1))
+    want[2, 5] += 1.5
+    assert np.array_equal(out, want)
+
+
 # ---------------------------------------------------------------- LayerNorm / GELU
 
 def test_layernorm_moments_and_affine():
