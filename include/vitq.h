@@ -86,6 +86,33 @@ typedef struct {
   vitq_merger_weights mergers[4];
 } vitq_tower_weights;
 
+/* bf16 variants ([FRT] s4: a massive-activation channel makes the image
+ * embeddings sensitive to FP8, so the first three blocks and the mergers keep
+ * bf16 weights and activations).  Same layout as above with bf16 weight
+ * matrices [out, in] instead of FP8 codes and scales. */
+typedef struct {
+  const void* norm1_w; const void* norm1_b;  /* [1152] */
+  const void* qkv_w; const void* qkv_b;      /* [3456,1152], [3456] */
+  const void* proj_w; const void* proj_b;    /* [1152,1152], [1152] */
+  const void* norm2_w; const void* norm2_b;  /* [1152] */
+  const void* fc1_w; const void* fc1_b;      /* [4304,1152], [4304] */
+  const void* fc2_w; const void* fc2_b;      /* [1152,4304], [1152] */
+} vitq_block_weights_bf16;
+
+typedef struct {
+  const void* norm_w; const void* norm_b;    /* [4608] */
+  const void* fc1_w; const void* fc1_b;      /* [4608,4608], [4608] */
+  const void* fc2_w; const void* fc2_b;      /* [2048,4608], [2048] */
+} vitq_merger_weights_bf16;
+
+/* Mixed-precision tower: blocks 1-3 and the 4 mergers bf16, blocks 4-27 FP8. */
+#define VITQ_BF16_HEAD_BLOCKS 3
+typedef struct {
+  vitq_block_weights_bf16 head[VITQ_BF16_HEAD_BLOCKS];
+  vitq_block_weights blocks[VITQ_BLOCKS - VITQ_BF16_HEAD_BLOCKS];
+  vitq_merger_weights_bf16 mergers[4];
+} vitq_tower_weights_mixed;
+
 /* ---------------------------------------------------------------- stages */
 
 /* 1x128 FP8 activation quantisation ([FRT] s3 "per-token / per-128-K-block FP8
@@ -219,6 +246,25 @@ int vit_merger_forward_static(const vitq_merger_weights* w, const void* x, int n
 int vit_tower_forward(const vitq_tower_weights* w, void* x, const int32_t* grid_hw, int n_images,
                       void* const* taps, void* ws, size_t ws_bytes, void* stream);
 size_t vitq_tower_workspace_bytes(int n_tokens_max, int n_images_max);
+
+/* bf16 block, in place on x bf16 [n_tokens, 1152]: LN1 (bf16) -> QKV bf16 GEMM +
+ * bias -> RoPE -> attention -> proj bf16 GEMM + bias + x -> LN2 (bf16) -> fc1
+ * bf16 GEMM + bias -> GELU (bf16) -> fc2 bf16 GEMM + bias + residual.  Arguments
+ * as vit_block_forward; ws >= vitq_block_workspace_bytes(n_tokens). */
+int vit_block_forward_bf16(const vitq_block_weights_bf16* w, void* x, int n_tokens, const int32_t* cu_seqlens,
+                           int n_seqs, int max_seqlen, const float* cos_sin, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* bf16 2x2 merger: as vit_merger_forward with bf16 LayerNorm output, bf16 fc1
+ * and fc2 and a bf16 GELU.  ws >= vitq_merger_bf16_workspace_bytes(n_tokens). */
+int vit_merger_forward_bf16(const vitq_merger_weights_bf16* w, const void* x, int n_tokens, void* out, void* ws,
+                            size_t ws_bytes, void* stream);
+size_t vitq_merger_bf16_workspace_bytes(int n_tokens);
+
+/* The tower with blocks 1-3 and the mergers in bf16 ([FRT] s4).  Arguments as
+ * vit_tower_forward; ws >= vitq_tower_workspace_bytes(n, n_images). */
+int vit_tower_forward_mixed(const vitq_tower_weights_mixed* w, void* x, const int32_t* grid_hw, int n_images,
+                            void* const* taps, void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------- status */
 

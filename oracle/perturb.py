@@ -11,11 +11,12 @@ fp64 rounding of every intermediate, so block-, merger- and tower-level outputs
 are compared against the drift the oracle itself shows when one of its
 intermediate roundings is moved by a tiny amount.
 
-Two perturbations are modelled, each a documented change of a rounding point:
+Three perturbations are modelled, each a documented change of a rounding point:
   gemm_fp32_promotion : the per-128-K partial sums (exact) are scaled and summed
                         in fp32 instead of fp64 (a ~1e-7 relative change);
   attention_bf16_p    : softmax probabilities rounded to bf16 before the P.V
-                        product, as a bf16 flash-attention kernel does.
+                        product, as a bf16 flash-attention kernel does;
+  bf16_gemm_fp32      : the bf16 GEMMs accumulate in fp32 instead of fp64.
 """
 from __future__ import annotations
 
@@ -63,12 +64,23 @@ def attention_bf16_p(qkv, cu_seqlens, heads: int = 16, head_dim: int = 72, scale
     return bf16_round(out.reshape(n, -1))
 
 
+def bf16_gemm_fp32(a, w, bias=None, residual=None):
+    """bf16_gemm with the product summed, and bias and residual added, in fp32."""
+    acc = np.asarray(a, np.float32) @ np.asarray(w, np.float32).T
+    if bias is not None:
+        acc = acc + np.asarray(bias, np.float32)[None, :]
+    if residual is not None:
+        acc = acc + np.asarray(residual, np.float32)
+    return bf16_round(acc.astype(np.float64))
+
+
 @contextlib.contextmanager
 def perturbed():
-    """Within the context, the oracle's block/merger/tower use both perturbations."""
-    g, a = ov.fp8_block_gemm, ov.attention_varlen
-    ov.fp8_block_gemm, ov.attention_varlen = fp8_block_gemm_fp32_promotion, attention_bf16_p
+    """Within the context, the oracle's block/merger/tower use the perturbations
+    (fp32 GEMM promotion or accumulation, bf16 attention probabilities)."""
+    g, a, b = ov.fp8_block_gemm, ov.attention_varlen, ov.bf16_gemm
+    ov.fp8_block_gemm, ov.attention_varlen, ov.bf16_gemm = fp8_block_gemm_fp32_promotion, attention_bf16_p, bf16_gemm_fp32
     try:
         yield
     finally:
-        ov.fp8_block_gemm, ov.attention_varlen = g, a
+        ov.fp8_block_gemm, ov.attention_varlen, ov.bf16_gemm = g, a, b

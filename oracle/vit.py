@@ -337,6 +337,37 @@ def block_forward(x, w: dict, cu_seqlens, pos, eps: float = 1e-6, keep: bool = F
     return (st["x2"], st) if keep else st["x2"]
 
 
+def block_forward_bf16(x, w: dict, cu_seqlens, pos, eps: float = 1e-6, keep: bool = False):
+    """One ViT block with bf16 linears [FRT s4: the first three blocks stay bf16]: LayerNorm and
+    GELU outputs rounded to bf16 and fed to bf16 GEMMs (no FP8 quantisation); w holds the
+    bf16-valued weights of block_params (qkv_w, proj_w, fc1_w, fc2_w [out, in]).
+    """
+    x = np.asarray(x, np.float64)
+    st = {}
+    st["h1"] = layernorm(x, w["norm1_w"], w["norm1_b"], eps)
+    st["qkv"] = bf16_gemm(st["h1"], w["qkv_w"], bias=w["qkv_b"])
+    st["qkv_rot"] = apply_rope_qkv(st["qkv"], pos)
+    st["attn"] = attention_varlen(st["qkv_rot"], cu_seqlens)
+    st["x1"] = bf16_gemm(st["attn"], w["proj_w"], bias=w["proj_b"], residual=x)
+    st["h2"] = layernorm(st["x1"], w["norm2_w"], w["norm2_b"], eps)
+    st["f"] = bf16_gemm(st["h2"], w["fc1_w"], bias=w["fc1_b"])
+    st["g"] = gelu_tanh(st["f"])
+    st["x2"] = bf16_gemm(st["g"], w["fc2_w"], bias=w["fc2_b"], residual=st["x1"])
+    return (st["x2"], st) if keep else st["x2"]
+
+
+def merger_forward_bf16(x, w: dict, eps: float = 1e-6, keep: bool = False):
+    """2x2 merger with bf16 linears [FRT s4: the mergers stay bf16]."""
+    x = np.asarray(x, np.float64)
+    n, c = x.shape
+    st = {}
+    st["h1"] = layernorm(x.reshape(n // 4, 4 * c), w["norm_w"], w["norm_b"], eps)
+    st["h"] = bf16_gemm(st["h1"], w["fc1_w"], bias=w["fc1_b"])
+    st["g"] = gelu_tanh(st["h"])
+    st["out"] = bf16_gemm(st["g"], w["fc2_w"], bias=w["fc2_b"])
+    return (st["out"], st) if keep else st["out"]
+
+
 def merger_forward(x, w: dict, eps: float = 1e-6, keep: bool = False):
     """2x2 merger: 4 consecutive rows -> one 4608 row, LayerNorm, fc1, GELU, fc2."""
     x = np.asarray(x, np.float64)
@@ -354,16 +385,18 @@ def tower_forward(x, blocks, mergers, grids, taps_after=(8, 16, 24, 27), eps: fl
                   on_block=None):
     """27 blocks over packed images, a merger after each tapped block.
 
-    blocks: list of quantised block weight dicts; mergers: list of 4 merger dicts.
+    blocks: list of block weight dicts, each either quantised (quantize_block_weights: FP8
+    block) or the bf16 weights themselves (no "qkv_q": bf16 block); mergers likewise.
     Returns the list of merger outputs (one per tap).
     """
     pos, cu = packed_positions(grids)
     h = np.asarray(x, np.float64)
     taps = []
     for b, w in enumerate(blocks, start=1):
-        h = block_forward(h, w, cu, pos, eps)
+        h = (block_forward if "qkv_q" in w else block_forward_bf16)(h, w, cu, pos, eps)
         if on_block is not None:
             on_block(b, h)
         if b in taps_after:
-            taps.append(merger_forward(h, mergers[taps_after.index(b)], eps))
+            m = mergers[taps_after.index(b)]
+            taps.append((merger_forward if "fc1_q" in m else merger_forward_bf16)(h, m, eps))
     return taps

@@ -164,6 +164,18 @@ MergerWs carve_merger(Carver& c, int n_tokens) {
   return w;
 }
 
+struct MergerBf16Ws {
+  __nv_bfloat16 *ln, *h;
+};
+
+MergerBf16Ws carve_merger_bf16(Carver& c, int n_tokens) {
+  const int m = n_tokens / 4;
+  MergerBf16Ws w;
+  w.ln = c.take<__nv_bfloat16>((size_t)m * VITQ_MERGE_IN * 2);
+  w.h = c.take<__nv_bfloat16>((size_t)m * VITQ_MERGE_IN * 2);
+  return w;
+}
+
 struct TowerWs {
   int32_t* pos;
   int32_t* cu;
@@ -286,6 +298,73 @@ int merger_impl(const vitq_merger_weights* w, const __nv_bfloat16* x, int n, __n
               launch_gelu_quant(m.h, rows, VITQ_MERGE_IN, VITQ_MERGE_IN, m.q, m.s, m.lds, num_sms, st));
   return gemm_checked(m.q, m.s, m.lds, w->fc2_q, w->fc2_s, w->fc2_b, nullptr, out, rows, VITQ_OUT_HIDDEN,
                       VITQ_MERGE_IN, num_sms, st);
+}
+
+bool block_bf16_weights_ok(const vitq_block_weights_bf16* w) {
+  const void* p[12] = {w ? w->norm1_w : nullptr, w ? w->norm1_b : nullptr, w ? w->qkv_w : nullptr,
+                       w ? w->qkv_b : nullptr,   w ? w->proj_w : nullptr,  w ? w->proj_b : nullptr,
+                       w ? w->norm2_w : nullptr, w ? w->norm2_b : nullptr, w ? w->fc1_w : nullptr,
+                       w ? w->fc1_b : nullptr,   w ? w->fc2_w : nullptr,   w ? w->fc2_b : nullptr};
+  for (const void* q : p)
+    if (!q || !al16(q)) return false;
+  return true;
+}
+
+bool merger_bf16_weights_ok(const vitq_merger_weights_bf16* w) {
+  const void* p[6] = {w ? w->norm_w : nullptr, w ? w->norm_b : nullptr, w ? w->fc1_w : nullptr,
+                      w ? w->fc1_b : nullptr,  w ? w->fc2_w : nullptr,  w ? w->fc2_b : nullptr};
+  for (const void* q : p)
+    if (!q || !al16(q)) return false;
+  return true;
+}
+
+// bf16 block: the LayerNorm outputs go to the codes region of the block
+// workspace (n * 4304 bytes >= n * 1152 bf16), GELU runs in place on the fc1 output.
+int block_bf16_impl(const vitq_block_weights_bf16* w, __nv_bfloat16* x, int n, const int32_t* cu, int n_seqs,
+                    int max_seqlen, const float* cs, const BlockWs& b, int num_sms, double attn_sumsq,
+                    cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  const double eps = 1e-6, dn = n;
+  bf* h = reinterpret_cast<bf*>(b.q);
+  const double ln_bytes = dn * VITQ_HIDDEN * 4;
+  VITQ_LAUNCH("ln_bf16", st, 0, ln_bytes,
+              launch_ln(x, VITQ_HIDDEN, (const bf*)w->norm1_w, (const bf*)w->norm1_b, n, VITQ_HIDDEN, eps, nullptr,
+                        nullptr, 0, h, st));
+  int r = bf16_gemm_checked(h, (const bf*)w->qkv_w, (const bf*)w->qkv_b, nullptr, b.qkv, n, VITQ_QKV,
+                            VITQ_HIDDEN, num_sms, st);
+  if (r) return r;
+  VITQ_LAUNCH("rope2d", st, 0, dn * 3456 * 2 * 2 + dn * 72 * 4, launch_rope_apply(b.qkv, n, cs, 1, st));
+  VITQ_LAUNCH("attention", st, 4.0 * attn_sumsq * VITQ_HEAD_DIM * VITQ_HEADS, dn * VITQ_QKV * 2 + dn * VITQ_HIDDEN * 2,
+              launch_attention(b.qkv, n, cu, n_seqs, max_seqlen, 1.0f / sqrtf((float)VITQ_HEAD_DIM), true, b.attn, st));
+  r = bf16_gemm_checked(b.attn, (const bf*)w->proj_w, (const bf*)w->proj_b, x, b.x1, n, VITQ_HIDDEN, VITQ_HIDDEN,
+                        num_sms, st);
+  if (r) return r;
+  VITQ_LAUNCH("ln_bf16", st, 0, ln_bytes,
+              launch_ln(b.x1, VITQ_HIDDEN, (const bf*)w->norm2_w, (const bf*)w->norm2_b, n, VITQ_HIDDEN, eps,
+                        nullptr, nullptr, 0, h, st));
+  r = bf16_gemm_checked(h, (const bf*)w->fc1_w, (const bf*)w->fc1_b, nullptr, b.f, n, VITQ_MLP, VITQ_HIDDEN,
+                        num_sms, st);
+  if (r) return r;
+  VITQ_LAUNCH("gelu_bf16", st, 0, dn * VITQ_MLP * 4,
+              launch_gelu(b.f, n, VITQ_MLP, VITQ_MLP, nullptr, nullptr, 0, b.f, num_sms, st));
+  return bf16_gemm_checked(b.f, (const bf*)w->fc2_w, (const bf*)w->fc2_b, b.x1, x, n, VITQ_HIDDEN, VITQ_MLP,
+                           num_sms, st);
+}
+
+int merger_bf16_impl(const vitq_merger_weights_bf16* w, const __nv_bfloat16* x, int n, __nv_bfloat16* out,
+                     const MergerBf16Ws& m, int num_sms, cudaStream_t st) {
+  using bf = __nv_bfloat16;
+  const int rows = n / 4;
+  VITQ_LAUNCH("ln_bf16", st, 0, (double)rows * VITQ_MERGE_IN * 4,
+              launch_ln(x, VITQ_MERGE_IN, (const bf*)w->norm_w, (const bf*)w->norm_b, rows, VITQ_MERGE_IN, 1e-6,
+                        nullptr, nullptr, 0, m.ln, st));
+  int r = bf16_gemm_checked(m.ln, (const bf*)w->fc1_w, (const bf*)w->fc1_b, nullptr, m.h, rows, VITQ_MERGE_IN,
+                            VITQ_MERGE_IN, num_sms, st);
+  if (r) return r;
+  VITQ_LAUNCH("gelu_bf16", st, 0, (double)rows * VITQ_MERGE_IN * 4,
+              launch_gelu(m.h, rows, VITQ_MERGE_IN, VITQ_MERGE_IN, nullptr, nullptr, 0, m.h, num_sms, st));
+  return bf16_gemm_checked(m.h, (const bf*)w->fc2_w, (const bf*)w->fc2_b, nullptr, out, rows, VITQ_OUT_HIDDEN,
+                           VITQ_MERGE_IN, num_sms, st);
 }
 
 }  // namespace
@@ -497,7 +576,11 @@ size_t vitq_tower_workspace_bytes(int n_tokens_max, int n_images_max) {
   carve_block(b, n_tokens_max);
   Carver m{nullptr};
   carve_merger(m, n_tokens_max);
-  return c.used + (b.used > m.used ? b.used : m.used);
+  Carver mb{nullptr};
+  carve_merger_bf16(mb, n_tokens_max);
+  size_t scratch = b.used > m.used ? b.used : m.used;
+  if (mb.used > scratch) scratch = mb.used;
+  return c.used + scratch;
 }
 
 int vit_block_forward(const vitq_block_weights* w, void* x, int n_tokens, const int32_t* cu_seqlens, int n_seqs,
@@ -532,13 +615,17 @@ int vit_merger_forward(const vitq_merger_weights* w, const void* x, int n_tokens
   return merger_impl(w, (const __nv_bfloat16*)x, n_tokens, (__nv_bfloat16*)out, m, sms, S(stream));
 }
 
-int vit_tower_forward(const vitq_tower_weights* w, void* x, const int32_t* grid_hw, int n_images,
-                      void* const* taps, void* ws, size_t ws_bytes, void* stream) {
-  VITQ_CHECK(w && x && taps && ws, VITQ_ERR_INVALID_ARG);
-  for (int t = 0; t < 4; ++t) VITQ_CHECK(taps[t] && al16(taps[t]), taps[t] ? VITQ_ERR_ALIGN : VITQ_ERR_INVALID_ARG);
-  for (int b = 0; b < VITQ_BLOCKS; ++b)
-    VITQ_CHECK(block_weights_ok(&w->blocks[b]), VITQ_ERR_INVALID_ARG);
-  for (int t = 0; t < 4; ++t) VITQ_CHECK(merger_weights_ok(&w->mergers[t]), VITQ_ERR_INVALID_ARG);
+}  // extern "C"
+
+namespace vitq {
+namespace {
+
+// Tower driver: positions and rope table, then the 27 blocks with the 4 mergers
+// after blocks 8, 16, 24 and 27.  run_block(blk, ...) and run_merger(tap, ...)
+// pick each block's and merger's precision.
+template <class BlockFn, class MergerFn>
+int tower_drive(void* x, const int32_t* grid_hw, int n_images, void* const* taps, void* ws, size_t ws_bytes,
+                void* stream, BlockFn run_block, MergerFn run_merger) {
   GridList g;
   int n = 0, max_len = 0;
   int r = fill_grids(grid_hw, n_images, true, &g, &n, &max_len);
@@ -553,8 +640,7 @@ int vit_tower_forward(const vitq_tower_weights* w, void* x, const int32_t* grid_
   TowerWs t = carve_tower_head(c, n, n_images);
   Carver rest{reinterpret_cast<uint8_t*>(ws) + c.used};
   BlockWs b = carve_block(rest, n);
-  Carver rest2{reinterpret_cast<uint8_t*>(ws) + c.used};
-  MergerWs m = carve_merger(rest2, n);
+  uint8_t* merger_ws = reinterpret_cast<uint8_t*>(ws) + c.used;   // aliases the block scratch
   VITQ_LAUNCH("positions", st, 0, (double)n * 8, launch_positions(g, n, t.pos, t.cu, st));
   VITQ_LAUNCH("rope_table", st, 0, (double)n * (8 + 288), launch_rope_table(t.pos, n, 10000.0, t.cs, st));
   double sumsq = 0;
@@ -563,15 +649,102 @@ int vit_tower_forward(const vitq_tower_weights* w, void* x, const int32_t* grid_
   int tap = 0;
   __nv_bfloat16* h = (__nv_bfloat16*)x;
   for (int blk = 1; blk <= VITQ_BLOCKS; ++blk) {
-    r = block_impl(&w->blocks[blk - 1], h, n, t.cu, n_images, max_len, t.cs, b, sms, sumsq, st);
+    r = run_block(blk, h, n, t.cu, n_images, max_len, t.cs, b, sms, sumsq, st);
     if (r) return r;
     if (tap < 4 && blk == kTap[tap]) {
-      r = merger_impl(&w->mergers[tap], h, n, (__nv_bfloat16*)taps[tap], m, sms, st);
+      r = run_merger(tap, h, n, (__nv_bfloat16*)taps[tap], merger_ws, sms, st);
       if (r) return r;
       ++tap;
     }
   }
   return VITQ_OK;
+}
+
+}  // namespace
+}  // namespace vitq
+
+extern "C" {
+
+int vit_tower_forward(const vitq_tower_weights* w, void* x, const int32_t* grid_hw, int n_images,
+                      void* const* taps, void* ws, size_t ws_bytes, void* stream) {
+  VITQ_CHECK(w && x && taps && ws, VITQ_ERR_INVALID_ARG);
+  for (int t = 0; t < 4; ++t) VITQ_CHECK(taps[t] && al16(taps[t]), taps[t] ? VITQ_ERR_ALIGN : VITQ_ERR_INVALID_ARG);
+  for (int b = 0; b < VITQ_BLOCKS; ++b)
+    VITQ_CHECK(block_weights_ok(&w->blocks[b]), VITQ_ERR_INVALID_ARG);
+  for (int t = 0; t < 4; ++t) VITQ_CHECK(merger_weights_ok(&w->mergers[t]), VITQ_ERR_INVALID_ARG);
+  return tower_drive(
+      x, grid_hw, n_images, taps, ws, ws_bytes, stream,
+      [&](int blk, __nv_bfloat16* h, int n, const int32_t* cu, int ni, int ml, const float* cs, const BlockWs& b,
+          int sms, double sumsq, cudaStream_t st) {
+        return block_impl(&w->blocks[blk - 1], h, n, cu, ni, ml, cs, b, sms, sumsq, st);
+      },
+      [&](int tap, const __nv_bfloat16* h, int n, __nv_bfloat16* out, uint8_t* mws, int sms, cudaStream_t st) {
+        Carver c{mws};
+        return merger_impl(&w->mergers[tap], h, n, out, carve_merger(c, n), sms, st);
+      });
+}
+
+int vit_tower_forward_mixed(const vitq_tower_weights_mixed* w, void* x, const int32_t* grid_hw, int n_images,
+                            void* const* taps, void* ws, size_t ws_bytes, void* stream) {
+  VITQ_CHECK(w && x && taps && ws, VITQ_ERR_INVALID_ARG);
+  for (int t = 0; t < 4; ++t) VITQ_CHECK(taps[t] && al16(taps[t]), taps[t] ? VITQ_ERR_ALIGN : VITQ_ERR_INVALID_ARG);
+  for (int b = 0; b < VITQ_BF16_HEAD_BLOCKS; ++b) VITQ_CHECK(block_bf16_weights_ok(&w->head[b]), VITQ_ERR_INVALID_ARG);
+  for (int b = 0; b < VITQ_BLOCKS - VITQ_BF16_HEAD_BLOCKS; ++b)
+    VITQ_CHECK(block_weights_ok(&w->blocks[b]), VITQ_ERR_INVALID_ARG);
+  for (int t = 0; t < 4; ++t) VITQ_CHECK(merger_bf16_weights_ok(&w->mergers[t]), VITQ_ERR_INVALID_ARG);
+  return tower_drive(
+      x, grid_hw, n_images, taps, ws, ws_bytes, stream,
+      [&](int blk, __nv_bfloat16* h, int n, const int32_t* cu, int ni, int ml, const float* cs, const BlockWs& b,
+          int sms, double sumsq, cudaStream_t st) {
+        if (blk <= VITQ_BF16_HEAD_BLOCKS)
+          return block_bf16_impl(&w->head[blk - 1], h, n, cu, ni, ml, cs, b, sms, sumsq, st);
+        return block_impl(&w->blocks[blk - 1 - VITQ_BF16_HEAD_BLOCKS], h, n, cu, ni, ml, cs, b, sms, sumsq, st);
+      },
+      [&](int tap, const __nv_bfloat16* h, int n, __nv_bfloat16* out, uint8_t* mws, int sms, cudaStream_t st) {
+        Carver c{mws};
+        return merger_bf16_impl(&w->mergers[tap], h, n, out, carve_merger_bf16(c, n), sms, st);
+      });
+}
+
+int vit_block_forward_bf16(const vitq_block_weights_bf16* w, void* x, int n_tokens, const int32_t* cu_seqlens,
+                           int n_seqs, int max_seqlen, const float* cos_sin, void* ws, size_t ws_bytes,
+                           void* stream) {
+  VITQ_CHECK(block_bf16_weights_ok(w), w ? VITQ_ERR_ALIGN : VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(x && cu_seqlens && cos_sin && ws, VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(n_tokens >= 0 && n_seqs >= 0 && max_seqlen >= 0, VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(al16(x) && al16(ws), VITQ_ERR_ALIGN);
+  VITQ_CHECK(ws_bytes >= vitq_block_workspace_bytes(n_tokens), VITQ_ERR_WORKSPACE);
+  int sms = 0;
+  int r = current_device_ok(&sms);
+  if (r) return r;
+  if (n_tokens == 0) return VITQ_OK;
+  Carver c{reinterpret_cast<uint8_t*>(ws)};
+  BlockWs b = carve_block(c, n_tokens);
+  return block_bf16_impl(w, (__nv_bfloat16*)x, n_tokens, cu_seqlens, n_seqs, max_seqlen, cos_sin, b, sms, 0.0,
+                         S(stream));
+}
+
+size_t vitq_merger_bf16_workspace_bytes(int n_tokens) {
+  if (n_tokens < 0) return 0;
+  Carver c{nullptr};
+  carve_merger_bf16(c, n_tokens);
+  return c.used;
+}
+
+int vit_merger_forward_bf16(const vitq_merger_weights_bf16* w, const void* x, int n_tokens, void* out, void* ws,
+                            size_t ws_bytes, void* stream) {
+  VITQ_CHECK(merger_bf16_weights_ok(w), w ? VITQ_ERR_ALIGN : VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(x && out && ws && n_tokens >= 0, VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(n_tokens % 4 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(al16(x) && al16(out) && al16(ws), VITQ_ERR_ALIGN);
+  VITQ_CHECK(ws_bytes >= vitq_merger_bf16_workspace_bytes(n_tokens), VITQ_ERR_WORKSPACE);
+  int sms = 0;
+  int r = current_device_ok(&sms);
+  if (r) return r;
+  if (n_tokens == 0) return VITQ_OK;
+  Carver c{reinterpret_cast<uint8_t*>(ws)};
+  MergerBf16Ws m = carve_merger_bf16(c, n_tokens);
+  return merger_bf16_impl(w, (const __nv_bfloat16*)x, n_tokens, (__nv_bfloat16*)out, m, sms, S(stream));
 }
 
 int vitq_get_device_error(void* stream) {

@@ -136,7 +136,7 @@ template <int ITERS>
 __global__ void __launch_bounds__(32 * kLnRows, 3)
     ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx, const __nv_bfloat16* __restrict__ gamma,
                     const __nv_bfloat16* __restrict__ beta, int M, int K, double eps,
-                    uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+                    uint8_t* __restrict__ q, float* __restrict__ s, int lds, __nv_bfloat16* __restrict__ y) {
   __shared__ uint4 sg[ITERS * 32], sb[ITERS * 32];
   for (int i = threadIdx.x; i < ITERS * 32; i += blockDim.x) {
     const int col = lane_col(i >> 5, i & 31);
@@ -227,7 +227,14 @@ __global__ void __launch_bounds__(32 * kLnRows, 3)
         }
       }
     }
-    quant_store(v, ok, lane, row, col, K, q, s, lds);
+    if (y) {   // bf16 output (the bf16 blocks and mergers): values are already bf16
+      if (ok)
+        *reinterpret_cast<uint4*>(y + (size_t)row * K + col) =
+            make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                       pack_bf16x2(v[6], v[7]));
+    } else {
+      quant_store(v, ok, lane, row, col, K, q, s, lds);
+    }
   }
 }
 
@@ -257,8 +264,8 @@ constexpr size_t kGeluSmem = 65536 * 2;
 // Persistent: one CTA per SM copies the table into shared memory, then each warp
 // takes (row, 256-column step) items in turn (lane layout of lane_col).
 __global__ void __launch_bounds__(kGeluThreads, 1)
-    gelu_quant_kernel(const __nv_bfloat16* __restrict__ f, int M, int K, int ldf,
-                      uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+    gelu_quant_kernel(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* __restrict__ q,
+                      float* __restrict__ s, int lds, __nv_bfloat16* y) {
   extern __shared__ __align__(16) uint16_t lut[];
   {
     const uint4* src = reinterpret_cast<const uint4*>(g_gelu_table);
@@ -289,7 +296,14 @@ __global__ void __launch_bounds__(kGeluThreads, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = 0.f;
     }
-    quant_store(v, ok, lane, row, col, K, q, s, lds);
+    if (y) {   // bf16 output (may be f itself: each lane reads its 8 values before writing them)
+      if (ok)
+        *reinterpret_cast<uint4*>(y + (size_t)row * ldf + col) =
+            make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
+                       pack_bf16x2(v[6], v[7]));
+    } else {
+      quant_store(v, ok, lane, row, col, K, q, s, lds);
+    }
   }
 }
 
@@ -508,19 +522,19 @@ cudaError_t launch_quant_act(const __nv_bfloat16* x, int M, int K, int ldx, uint
 template <int IT>
 static void ln_launch(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* g,
                       const __nv_bfloat16* b, int M, int K, double eps, uint8_t* q, float* s, int lds,
-                      cudaStream_t st) {
+                      __nv_bfloat16* y, cudaStream_t st) {
   ln_quant_kernel<IT><<<(unsigned)((M + kLnRows - 1) / kLnRows), 32 * kLnRows, 0, st>>>(
-      x, ldx, g, b, M, K, eps, q, s, lds);
+      x, ldx, g, b, M, K, eps, q, s, lds, y);
 }
 
-cudaError_t launch_ln_quant(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma,
-                            const __nv_bfloat16* beta, int M, int K, double eps, uint8_t* q,
-                            float* s, int lds, cudaStream_t st) {
+cudaError_t launch_ln(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,
+                      int M, int K, double eps, uint8_t* q, float* s, int lds, __nv_bfloat16* y,
+                      cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   const int it = (K + 255) / 256;
   switch (it) {
 #define VITQ_LN_CASE(N) \
-  case N: ln_launch<N>(x, ldx, gamma, beta, M, K, eps, q, s, lds, st); break;
+  case N: ln_launch<N>(x, ldx, gamma, beta, M, K, eps, q, s, lds, y, st); break;
     VITQ_LN_CASE(1) VITQ_LN_CASE(2) VITQ_LN_CASE(3) VITQ_LN_CASE(4) VITQ_LN_CASE(5)
     VITQ_LN_CASE(6) VITQ_LN_CASE(7) VITQ_LN_CASE(8) VITQ_LN_CASE(9) VITQ_LN_CASE(10)
     VITQ_LN_CASE(11) VITQ_LN_CASE(12) VITQ_LN_CASE(13) VITQ_LN_CASE(14) VITQ_LN_CASE(15)
@@ -536,8 +550,8 @@ cudaError_t build_gelu_table(cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_gelu_quant(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* q, float* s,
-                              int lds, int num_sms, cudaStream_t st) {
+cudaError_t launch_gelu(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* q, float* s, int lds,
+                        __nv_bfloat16* y, int num_sms, cudaStream_t st) {
   if (M == 0) return cudaSuccess;
   cudaError_t e = cudaFuncSetAttribute(gelu_quant_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kGeluSmem);
@@ -545,7 +559,7 @@ cudaError_t launch_gelu_quant(const __nv_bfloat16* f, int M, int K, int ldf, uin
   const long long warps = (long long)M * ((K + 255) / 256);
   const long long ctas = (warps + kGeluThreads / 32 - 1) / (kGeluThreads / 32);
   gelu_quant_kernel<<<(unsigned)(ctas < num_sms ? ctas : num_sms), kGeluThreads, kGeluSmem, st>>>(
-      f, M, K, ldf, q, s, lds);
+      f, M, K, ldf, q, s, lds, y);
   return cudaGetLastError();
 }
 
@@ -579,4 +593,16 @@ cudaError_t launch_positions(const GridList& g, int n_total, int32_t* pos, int32
   return cudaGetLastError();
 }
 
+}  // namespace vitq
+
+namespace vitq {
+cudaError_t launch_ln_quant(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma,
+                            const __nv_bfloat16* beta, int M, int K, double eps, uint8_t* q,
+                            float* s, int lds, cudaStream_t st) {
+  return launch_ln(x, ldx, gamma, beta, M, K, eps, q, s, lds, nullptr, st);
+}
+cudaError_t launch_gelu_quant(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* q, float* s,
+                              int lds, int num_sms, cudaStream_t st) {
+  return launch_gelu(f, M, K, ldf, q, s, lds, nullptr, num_sms, st);
+}
 }  // namespace vitq

@@ -33,6 +33,12 @@ cudaError_t launch_quant_act(const __nv_bfloat16* x, int M, int K, int ldx, uint
 cudaError_t launch_ln_quant(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma,
                             const __nv_bfloat16* beta, int M, int K, double eps, uint8_t* q,
                             float* s, int lds, cudaStream_t st);
+// LayerNorm / GELU with either FP8 output (q, s) or bf16 output (y, when not null).
+cudaError_t launch_ln(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,
+                      int M, int K, double eps, uint8_t* q, float* s, int lds, __nv_bfloat16* y,
+                      cudaStream_t st);
+cudaError_t launch_gelu(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* q, float* s, int lds,
+                        __nv_bfloat16* y, int num_sms, cudaStream_t st);
 // One-time per device: GELU of every bf16 value into the device table.
 cudaError_t build_gelu_table(cudaStream_t st);
 cudaError_t launch_gelu_quant(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* q, float* s,

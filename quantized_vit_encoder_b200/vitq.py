@@ -39,6 +39,25 @@ class TowerWeights(C.Structure):
     _fields_ = [("blocks", BlockWeights * N_BLOCKS), ("mergers", MergerWeights * 4)]
 
 
+BF16_HEAD_BLOCKS = 3
+
+
+class BlockWeightsBf16(C.Structure):
+    _fields_ = [(n, _vp) for n in (
+        "norm1_w", "norm1_b", "qkv_w", "qkv_b", "proj_w", "proj_b",
+        "norm2_w", "norm2_b", "fc1_w", "fc1_b", "fc2_w", "fc2_b")]
+
+
+class MergerWeightsBf16(C.Structure):
+    _fields_ = [(n, _vp) for n in ("norm_w", "norm_b", "fc1_w", "fc1_b", "fc2_w", "fc2_b")]
+
+
+class TowerWeightsMixed(C.Structure):
+    _fields_ = [("head", BlockWeightsBf16 * BF16_HEAD_BLOCKS),
+                ("blocks", BlockWeights * (N_BLOCKS - BF16_HEAD_BLOCKS)),
+                ("mergers", MergerWeightsBf16 * 4)]
+
+
 _SIGS = {
     "vit_quant_act": [_vp, _i, _i, _i, _vp, _vp, _i, _vp],
     "vit_quant_weight": [_vp, _i, _i, _vp, _vp, _vp],
@@ -57,6 +76,10 @@ _SIGS = {
     "vitq_merger_workspace_bytes": [_i],
     "vit_tower_forward": [C.POINTER(TowerWeights), _vp, _vp, _i, C.POINTER(_vp), _vp, _sz, _vp],
     "vitq_tower_workspace_bytes": [_i, _i],
+    "vit_block_forward_bf16": [C.POINTER(BlockWeightsBf16), _vp, _i, _vp, _i, _i, _vp, _vp, _sz, _vp],
+    "vit_merger_forward_bf16": [C.POINTER(MergerWeightsBf16), _vp, _i, _vp, _vp, _sz, _vp],
+    "vitq_merger_bf16_workspace_bytes": [_i],
+    "vit_tower_forward_mixed": [C.POINTER(TowerWeightsMixed), _vp, _vp, _i, C.POINTER(_vp), _vp, _sz, _vp],
     "vitq_get_device_error": [_vp],
     "vitq_status_string": [_i],
     "vitq_launch_count": [],
@@ -67,6 +90,7 @@ _SIGS = {
     "vitq_selftest_wait_timeout": [_i, _vp],
 }
 _RES = {"vitq_block_workspace_bytes": _sz, "vitq_merger_workspace_bytes": _sz,
+        "vitq_merger_bf16_workspace_bytes": _sz,
         "vitq_tower_workspace_bytes": _sz, "vitq_status_string": C.c_char_p,
         "vitq_launch_count": C.c_ulonglong, "vitq_profile_start": None}
 
@@ -258,6 +282,67 @@ class DeviceMerger:
         for name in ("fc1", "fc2"):
             t[name + "_q"], t[name + "_s"] = quant_weight(t[name + "_w"], stream)
         self.struct = MergerWeights(**{f: t[f].data_ptr() for f, _ in MergerWeights._fields_})
+
+
+class DeviceBlockBf16:
+    """Device-resident bf16 block weights (no quantisation) and their C struct."""
+
+    def __init__(self, params: dict, device="cuda"):
+        self.t = {k: v.to(device).contiguous() for k, v in params.items()}
+        self.struct = BlockWeightsBf16(**{f: self.t[f].data_ptr() for f, _ in BlockWeightsBf16._fields_})
+
+
+class DeviceMergerBf16:
+    def __init__(self, params: dict, device="cuda"):
+        self.t = {k: v.to(device).contiguous() for k, v in params.items()}
+        self.struct = MergerWeightsBf16(**{f: self.t[f].data_ptr() for f, _ in MergerWeightsBf16._fields_})
+
+
+class DeviceTowerMixed:
+    """Blocks 1-3 and the mergers bf16 (DeviceBlockBf16 / DeviceMergerBf16), blocks 4-27 FP8 (DeviceBlock)."""
+
+    def __init__(self, head, blocks, mergers):
+        self.head, self.blocks, self.mergers = head, blocks, mergers
+        self.struct = TowerWeightsMixed()
+        for i, b in enumerate(head):
+            self.struct.head[i] = b.struct
+        for i, b in enumerate(blocks):
+            self.struct.blocks[i] = b.struct
+        for i, m in enumerate(mergers):
+            self.struct.mergers[i] = m.struct
+
+
+def block_forward_bf16_(blk: DeviceBlockBf16, x, cu_seqlens, max_seqlen, cos_sin, ws, stream=None):
+    """In-place bf16 block forward on bf16 x [n, 1152]."""
+    _check(load().vit_block_forward_bf16(C.byref(blk.struct), _p(x), x.shape[0], _p(cu_seqlens),
+                                         cu_seqlens.shape[0] - 1, max_seqlen, _p(cos_sin), _p(ws), ws.numel(),
+                                         _stream(stream)), "vit_block_forward_bf16")
+    return x
+
+
+def merger_bf16_workspace_bytes(n: int) -> int:
+    return int(load().vitq_merger_bf16_workspace_bytes(n))
+
+
+def merger_forward_bf16(mg: DeviceMergerBf16, x, ws, out=None, stream=None):
+    n = x.shape[0]
+    if out is None:
+        out = torch.empty((n // 4, OUT_HIDDEN), dtype=torch.bfloat16, device=x.device)
+    _check(load().vit_merger_forward_bf16(C.byref(mg.struct), _p(x), n, _p(out), _p(ws), ws.numel(),
+                                          _stream(stream)), "vit_merger_forward_bf16")
+    return out
+
+
+def tower_forward_mixed_(tower: DeviceTowerMixed, x, grids, ws, taps=None, stream=None):
+    """In-place mixed-precision tower forward; returns the four taps [n/4, 2048]."""
+    n = x.shape[0]
+    if taps is None:
+        taps = [torch.empty((n // 4, OUT_HIDDEN), dtype=torch.bfloat16, device=x.device) for _ in range(4)]
+    g = (C.c_int32 * (2 * len(grids)))(*[v for hw in grids for v in hw])
+    tp = (C.c_void_p * 4)(*[t.data_ptr() for t in taps])
+    _check(load().vit_tower_forward_mixed(C.byref(tower.struct), _p(x), C.cast(g, C.c_void_p), len(grids), tp,
+                                          _p(ws), ws.numel(), _stream(stream)), "vit_tower_forward_mixed")
+    return taps
 
 
 def block_workspace_bytes(n: int) -> int:

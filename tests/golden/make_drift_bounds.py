@@ -65,7 +65,45 @@ def tower_case(grids, scales, seed_base):
     return [stats(a, r) for a, r in zip(alt, ref)]
 
 
+def block_bf16_case(name):
+    W = wl.WORKLOADS[name]
+    x = f64(wl.make_input(W))
+    w = {k: f64(v) for k, v in wl.block_params(wl.block_seed(W, 0)).items()}
+    pos, cu = ov.packed_positions(W.grids)
+    ref = ov.block_forward_bf16(x, w, cu, pos)
+    with perturb.perturbed():
+        alt = ov.block_forward_bf16(x, w, cu, pos)
+    return stats(alt, ref)
+
+
+def merger_bf16_case(n):
+    x = f64(wl.random_bf16((n, 1152), 700 + n, 2.0))
+    m = {k: f64(v) for k, v in wl.merger_params(4242).items()}
+    ref = ov.merger_forward_bf16(x, m)
+    with perturb.perturbed():
+        alt = ov.merger_forward_bf16(x, m)
+    return stats(alt, ref)
+
+
+def tower_mixed_case(grids, scales, seed_base):
+    W = wl.Workload("tower_case", tuple(grids), wl.N_BLOCKS, True, scales=tuple(scales), seed_base=seed_base)
+    x = f64(wl.make_input(W))
+    blocks = []
+    for b in range(wl.N_BLOCKS):
+        p = {k: f64(v) for k, v in wl.block_params(wl.block_seed(W, b)).items()}
+        blocks.append(p if b < 3 else ov.quantize_block_weights(p))
+    mergers = [{k: f64(v) for k, v in wl.merger_params(wl.merger_seed(W, t)).items()} for t in range(4)]
+    ref = ov.tower_forward(x, blocks, mergers, W.grids)
+    with perturb.perturbed():
+        alt = ov.tower_forward(x, blocks, mergers, W.grids)
+    return [stats(a, r) for a, r in zip(alt, ref)]
+
+
 CASES = {
+    "block_bf16_16x16": lambda: block_bf16_case("block_16x16"),
+    "block_bf16_36x27": lambda: block_bf16_case("block_36x27"),
+    "merger_bf16_972": lambda: merger_bf16_case(972),
+    "tower_mixed_small": lambda: tower_mixed_case([(16, 16), (8, 12)], [1.0, 3.0], 5200),
     "block_16x16": lambda: block_case("block_16x16"),
     "block_36x27": lambda: block_case("block_36x27"),
     "block_46x136": lambda: block_case("block_46x136"),
