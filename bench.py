@@ -329,6 +329,37 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     barrier()
     block_ms = max_over_ranks(ev0.elapsed_time(ev1) / nb)
 
+    # bf16 variant of the block and the mixed-precision tower (blocks 1-3 and mergers bf16)
+    bkeys = [f for f, _ in vitq.BlockWeightsBf16._fields_]
+    mkeys = [f for f, _ in vitq.MergerWeightsBf16._fields_]
+    head = [vitq.DeviceBlockBf16({k: tower.blocks[b].t[k] for k in bkeys}, dev) for b in range(vitq.BF16_HEAD_BLOCKS)]
+    mixed = vitq.DeviceTowerMixed(head, tower.blocks[vitq.BF16_HEAD_BLOCKS:],
+                                  [vitq.DeviceMergerBf16({k: m.t[k] for k in mkeys}, dev) for m in tower.mergers])
+    xb.copy_(x0)
+    for _ in range(args.warmup):
+        vitq.block_forward_bf16_(head[0], xb, cu, W.n_tokens, cs, wsb)
+    barrier()
+    ev0.record(stream)
+    for _ in range(nb):
+        vitq.block_forward_bf16_(head[0], xb, cu, W.n_tokens, cs, wsb)
+    ev1.record(stream)
+    barrier()
+    block_bf16_ms = max_over_ranks(ev0.elapsed_time(ev1) / nb)
+
+    def mixed_step():
+        x.copy_(x0, non_blocking=True)
+        vitq.tower_forward_mixed_(mixed, x, grids, ws, taps)
+
+    for _ in range(args.warmup):
+        mixed_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        mixed_step()
+    ev1.record(stream)
+    barrier()
+    mixed_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+
     # per-kernel device times from a profiled pass of the same step (not the timed one)
     vitq.profile_start()
     for _ in range(2):
@@ -379,6 +410,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "block_frac_of_peak": ideal_block_ms / block_ms,
         "block_ideal_ms": ideal_block_ms,
         "tower_ms": ms,
+        "block_bf16_ms": block_bf16_ms,
+        "mixed_tower_ms": mixed_ms,
         "roofline": roofline(table, peaks),
         "kernels": {k: {"launches": v["launches"] // 2, "ms_per_step": v["ms"] / 2,
                         "share": v["ms"] / sum(t["ms"] for t in table.values())} for k, v in table.items()},

@@ -132,7 +132,7 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ x, int M, int
 
 constexpr int kLnRows = 8;
 
-template <int ITERS>
+template <int ITERS, bool kOutBf16>
 __global__ void __launch_bounds__(32 * kLnRows, 3)
     ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx, const __nv_bfloat16* __restrict__ gamma,
                     const __nv_bfloat16* __restrict__ beta, int M, int K, double eps,
@@ -227,7 +227,7 @@ __global__ void __launch_bounds__(32 * kLnRows, 3)
         }
       }
     }
-    if (y) {   // bf16 output (the bf16 blocks and mergers): values are already bf16
+    if (kOutBf16) {   // bf16 output (the bf16 blocks and mergers): values are already bf16
       if (ok)
         *reinterpret_cast<uint4*>(y + (size_t)row * K + col) =
             make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
@@ -523,8 +523,12 @@ template <int IT>
 static void ln_launch(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* g,
                       const __nv_bfloat16* b, int M, int K, double eps, uint8_t* q, float* s, int lds,
                       __nv_bfloat16* y, cudaStream_t st) {
-  ln_quant_kernel<IT><<<(unsigned)((M + kLnRows - 1) / kLnRows), 32 * kLnRows, 0, st>>>(
-      x, ldx, g, b, M, K, eps, q, s, lds, y);
+  if (y)
+    ln_quant_kernel<IT, true><<<(unsigned)((M + kLnRows - 1) / kLnRows), 32 * kLnRows, 0, st>>>(
+        x, ldx, g, b, M, K, eps, q, s, lds, y);
+  else
+    ln_quant_kernel<IT, false><<<(unsigned)((M + kLnRows - 1) / kLnRows), 32 * kLnRows, 0, st>>>(
+        x, ldx, g, b, M, K, eps, q, s, lds, y);
 }
 
 cudaError_t launch_ln(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,

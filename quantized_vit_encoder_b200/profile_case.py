@@ -2,8 +2,8 @@
 
     python -m quantized_vit_encoder_b200.profile_case STAGE [--iters N]
 
-STAGE: attention | gemm_qkv | gemm_proj | gemm_fc1 | gemm_fc2 | ln_quant | ln_quant_merger |
-       quant_act | gelu_quant | rope | block.
+STAGE: attention | gemm_qkv | gemm_proj | gemm_fc1 | gemm_fc2 | bf16_qkv | bf16_proj | bf16_fc1 |
+       bf16_fc2 | ln_quant | ln_quant_merger | quant_act | gelu_quant | rope | block.
 Device memory stays below 0.5 GB; each iteration is one launch of the stage's
 kernel (block: the ten launches of one block).
 """
@@ -49,6 +49,12 @@ def main():
         res = x if name in ("proj",) else (wl.random_bf16((n, 1152), 3).to(dev) if name == "fc2" else None)
         out = torch.empty((n, w.shape[0]), dtype=torch.bfloat16, device=dev)
         run = lambda: vitq.fp8_block_gemm(qa, sa, t[name + "_q"], t[name + "_s"], t[name + "_b"], res, out)  # noqa: E731
+    elif a.stage.startswith("bf16_"):
+        name = a.stage[5:]
+        w = t[name + "_w"]
+        act = wl.random_bf16((n, w.shape[1]), 2, 1.0).to(dev)
+        out = torch.empty((n, w.shape[0]), dtype=torch.bfloat16, device=dev)
+        run = lambda: vitq.bf16_gemm(act, w, t[name + "_b"], None, out)  # noqa: E731
     elif a.stage == "ln_quant":
         run = lambda: vitq.ln_quant(x, t["norm1_w"], t["norm1_b"])  # noqa: E731
     elif a.stage == "ln_quant_merger":
