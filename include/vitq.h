@@ -195,6 +195,23 @@ int vit_positions(const int32_t* grid_hw, int n_images, int32_t* pos_hw, int32_t
 int vit_attention_varlen(const void* qkv, int n_tokens, const int32_t* cu_seqlens, int n_seqs,
                          int max_seqlen, float softmax_scale, int flags, void* out, void* stream);
 
+/* Patch embedding with the interpolated position embedding ([FRT] s3
+ * "patch_embed -> +interpolated pos_embed"; [VE] PATCH_DIM = 3*2*16*16 = 1536,
+ * patch_embed_w [1152, 1536], pos_embed [2304, 1152], num_grid_per_side 48):
+ *   x[t] = bf16( pixels[t] . w^T + b + pos[t] ),
+ * pos[t] = bf16(bilinear interpolation of the 48 x 48 table at the token's
+ * (row, col)), sample points running corner to corner (row r of an h-row grid
+ * at table row r * 47 / (h - 1)).  pixels: bf16 [n_tokens, 1536], patchified,
+ * in the tower's token order (see vit_positions); grid_hw: HOST int32
+ * [n_images][2] with sum h*w == n_tokens (any h, w); w bf16 [1152, 1536];
+ * b bf16 [1152]; pos_table bf16 [2304, 1152]; x bf16 [n_tokens, 1152] (output).
+ * ws >= vitq_patch_embed_workspace_bytes(n_tokens).  All 16-byte aligned. */
+int vit_patch_embed(const void* pixels, int n_tokens, const int32_t* grid_hw, int n_images, const void* w,
+                    const void* b, const void* pos_table, void* x, void* ws, size_t ws_bytes, void* stream);
+size_t vitq_patch_embed_workspace_bytes(int n_tokens);
+#define VITQ_PATCH_DIM 1536
+#define VITQ_POS_GRID 48
+
 /* ---------------------------------------------------------------- layers */
 
 /* One ViT block in place on x bf16 [n_tokens, 1152] ([FRT] s3 per-block chain):

@@ -227,6 +227,50 @@ def packed_positions(grids) -> tuple:
     return np.concatenate(pos, 0), np.asarray(cu, np.int64)
 
 
+# --------------------------------------------------------------------------
+# Patch embedding and interpolated position embedding
+# [FRT s3 "patch_embed -> +interpolated pos_embed"; VE PATCH_DIM = 3*2*16*16 = 1536,
+#  patch_embed_w [1152, 1536], pos_embed [2304, 1152], num_grid_per_side 48]
+# --------------------------------------------------------------------------
+
+POS_GRID = 48
+
+
+def pos_embed_interp(table, h: int, w: int) -> np.ndarray:
+    """Bilinear interpolation of the learned 48 x 48 position table to an h x w patch grid.
+
+    Sample points run from corner to corner: grid row r of h sits at table row
+    r * 47 / (h - 1) (0 when h = 1), likewise for columns; each value mixes the
+    four surrounding table entries with the usual bilinear weights.  fp64,
+    not rounded: [h, w, C].
+    """
+    T = np.asarray(table, np.float64).reshape(POS_GRID, POS_GRID, -1)
+    fy = np.arange(h, dtype=np.float64) * ((POS_GRID - 1) / (h - 1) if h > 1 else 0.0)
+    fx = np.arange(w, dtype=np.float64) * ((POS_GRID - 1) / (w - 1) if w > 1 else 0.0)
+    y0 = np.floor(fy).astype(np.int64)
+    x0 = np.floor(fx).astype(np.int64)
+    y1 = np.minimum(y0 + 1, POS_GRID - 1)
+    x1 = np.minimum(x0 + 1, POS_GRID - 1)
+    dy = (fy - y0)[:, None, None]
+    dx = (fx - x0)[None, :, None]
+    return ((1 - dy) * (1 - dx) * T[y0][:, x0] + (1 - dy) * dx * T[y0][:, x1]
+            + dy * (1 - dx) * T[y1][:, x0] + dy * dx * T[y1][:, x1])
+
+
+def patch_embed(pixels, w, b, table, grids) -> np.ndarray:
+    """x = bf16( pixels @ w^T + b + pos ) over packed images in token order, where pos is
+    the interpolated position embedding of each patch rounded to bf16.
+
+    pixels: [n, 1536] patch rows (already normalised and patchified); w [1152, 1536].
+    """
+    pos = []
+    for h, wd in grids:
+        grid = pos_embed_interp(table, h, wd)
+        rc = patch_positions(h, wd)
+        pos.append(grid[rc[:, 0], rc[:, 1]])
+    return bf16_gemm(pixels, w, bias=b, residual=bf16_round(np.concatenate(pos, 0)))
+
+
 def rope_inv_freq(head_dim: int = 72, theta: float = 10000.0) -> np.ndarray:
     """head_dim/4 frequencies theta**(-2i/(head_dim/2)), fp64."""
     half = head_dim // 2

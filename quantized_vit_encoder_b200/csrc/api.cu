@@ -724,6 +724,33 @@ int vit_block_forward_bf16(const vitq_block_weights_bf16* w, void* x, int n_toke
                          S(stream));
 }
 
+size_t vitq_patch_embed_workspace_bytes(int n_tokens) {
+  if (n_tokens < 0) return 0;
+  return up256((size_t)n_tokens * VITQ_HIDDEN * 2);
+}
+
+int vit_patch_embed(const void* pixels, int n_tokens, const int32_t* grid_hw, int n_images, const void* w,
+                    const void* b, const void* pos_table, void* x, void* ws, size_t ws_bytes, void* stream) {
+  VITQ_CHECK(pixels && w && b && pos_table && x && ws && n_tokens >= 0, VITQ_ERR_INVALID_ARG);
+  GridList g;
+  int n = 0, max_len = 0;
+  int r = fill_grids(grid_hw, n_images, false, &g, &n, &max_len);
+  if (r) return r;
+  VITQ_CHECK(n == n_tokens, VITQ_ERR_SHAPE);
+  VITQ_CHECK(al16(pixels) && al16(w) && al16(b) && al16(pos_table) && al16(x) && al16(ws), VITQ_ERR_ALIGN);
+  VITQ_CHECK(ws_bytes >= vitq_patch_embed_workspace_bytes(n_tokens), VITQ_ERR_WORKSPACE);
+  int sms = 0;
+  r = current_device_ok(&sms);
+  if (r) return r;
+  if (n_tokens == 0) return VITQ_OK;
+  cudaStream_t st = S(stream);
+  __nv_bfloat16* pos = reinterpret_cast<__nv_bfloat16*>(ws);
+  VITQ_LAUNCH("pos_interp", st, 0, (double)n_tokens * VITQ_HIDDEN * (4 * 2 + 2),
+              launch_pos_interp(g, n_tokens, (const __nv_bfloat16*)pos_table, pos, st));
+  return bf16_gemm_checked((const __nv_bfloat16*)pixels, (const __nv_bfloat16*)w, (const __nv_bfloat16*)b, pos,
+                           (__nv_bfloat16*)x, n_tokens, VITQ_HIDDEN, VITQ_PATCH_DIM, sms, st);
+}
+
 size_t vitq_merger_bf16_workspace_bytes(int n_tokens) {
   if (n_tokens < 0) return 0;
   Carver c{nullptr};

@@ -435,6 +435,65 @@ __global__ void __launch_bounds__(432) rope_apply_kernel(__nv_bfloat16* __restri
 // Token order inside an h x w image: 2x2-block order for even grids (block
 // (br, bc) row-major, inside it (0,0) (0,1) (1,0) (1,1)), row-major otherwise.
 
+// Image of token t of the packed images, and the token's (row, col) in that image:
+// 2x2-block order (merger neighbours consecutive) for even grids, row-major otherwise.
+__device__ __forceinline__ void token_place(const GridList& grids, int t, int& img, int& r, int& c) {
+  int start = 0;
+  for (img = 0; img < grids.n - 1; ++img) {
+    const int len = grids.hw[2 * img] * grids.hw[2 * img + 1];
+    if (t < start + len) break;
+    start += len;
+  }
+  const int h = grids.hw[2 * img], w = grids.hw[2 * img + 1];
+  const int p = t - start;
+  if ((h & 1) == 0 && (w & 1) == 0) {
+    const int blk = p >> 2, within = p & 3;
+    const int br = blk / (w >> 1), bc = blk - br * (w >> 1);
+    r = 2 * br + (within >> 1);
+    c = 2 * bc + (within & 1);
+  } else {
+    r = p / w;
+    c = p - r * w;
+  }
+}
+
+// ------------------------------------------------- interpolated position embedding
+// "Qwen3-VL-8B on RTX 5090", section 3 (patch_embed -> + interpolated pos_embed):
+// the learned 48 x 48 table is interpolated bilinearly to each image's patch grid,
+// sample points running corner to corner (row r of h at r * 47 / (h - 1)).  fp64
+// weights and sums of the bf16 table values, rounded once to bf16.  One CTA of 144
+// threads per token, 8 channels per thread.
+constexpr int kPosGrid = 48;
+
+__global__ void __launch_bounds__(144) pos_interp_kernel(GridList grids, const __nv_bfloat16* __restrict__ table,
+                                                         __nv_bfloat16* __restrict__ out) {
+  const int t = blockIdx.x;
+  int img, r, c;
+  token_place(grids, t, img, r, c);
+  const int h = grids.hw[2 * img], w = grids.hw[2 * img + 1];
+  const double fy = (double)r * (h > 1 ? (double)(kPosGrid - 1) / (double)(h - 1) : 0.0);
+  const double fx = (double)c * (w > 1 ? (double)(kPosGrid - 1) / (double)(w - 1) : 0.0);
+  const int y0 = (int)floor(fy), x0 = (int)floor(fx);
+  const int y1 = min(y0 + 1, kPosGrid - 1), x1 = min(x0 + 1, kPosGrid - 1);
+  const double dy = fy - y0, dx = fx - x0;
+  const double w00 = (1 - dy) * (1 - dx), w01 = (1 - dy) * dx, w10 = dy * (1 - dx), w11 = dy * dx;
+  const int d0 = threadIdx.x * 8;
+  float v00[8], v01[8], v10[8], v11[8];
+  load8_bf16(table + (size_t)(y0 * kPosGrid + x0) * 1152 + d0, v00);
+  load8_bf16(table + (size_t)(y0 * kPosGrid + x1) * 1152 + d0, v01);
+  load8_bf16(table + (size_t)(y1 * kPosGrid + x0) * 1152 + d0, v10);
+  load8_bf16(table + (size_t)(y1 * kPosGrid + x1) * 1152 + d0, v11);
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const double a = w00 * v00[2 * i] + w01 * v01[2 * i] + w10 * v10[2 * i] + w11 * v11[2 * i];
+    const double b = w00 * v00[2 * i + 1] + w01 * v01[2 * i + 1] + w10 * v10[2 * i + 1] + w11 * v11[2 * i + 1];
+    const __nv_bfloat16 ha = __double2bfloat16(a), hb = __double2bfloat16(b);
+    o[i] = (uint32_t)__bfloat16_as_ushort(ha) | ((uint32_t)__bfloat16_as_ushort(hb) << 16);
+  }
+  *reinterpret_cast<uint4*>(out + (size_t)t * 1152 + d0) = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 __global__ void positions_kernel(GridList grids, int n_total, int32_t* __restrict__ pos,
                                  int32_t* __restrict__ cu) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -447,24 +506,8 @@ __global__ void positions_kernel(GridList grids, int n_total, int32_t* __restric
     }
   }
   if (t >= n_total) return;
-  int start = 0, img = 0;
-  for (; img < grids.n; ++img) {
-    const int len = grids.hw[2 * img] * grids.hw[2 * img + 1];
-    if (t < start + len) break;
-    start += len;
-  }
-  const int h = grids.hw[2 * img], w = grids.hw[2 * img + 1];
-  const int p = t - start;
-  int r, c;
-  if ((h & 1) == 0 && (w & 1) == 0) {
-    const int blk = p >> 2, within = p & 3;
-    const int br = blk / (w >> 1), bc = blk - br * (w >> 1);
-    r = 2 * br + (within >> 1);
-    c = 2 * bc + (within & 1);
-  } else {
-    r = p / w;
-    c = p - r * w;
-  }
+  int img, r, c;
+  token_place(grids, t, img, r, c);
   pos[2 * t] = r;
   pos[2 * t + 1] = c;
 }
@@ -586,6 +629,13 @@ cudaError_t launch_rope_table(const int32_t* pos, int n, double theta, float* cs
 cudaError_t launch_rope_apply(__nv_bfloat16* qkv, int n, const float* cs, int v_to_f16, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   rope_apply_kernel<<<n, 432, 0, st>>>(qkv, cs, v_to_f16);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pos_interp(const GridList& g, int n_total, const __nv_bfloat16* table, __nv_bfloat16* out,
+                              cudaStream_t st) {
+  if (n_total == 0) return cudaSuccess;
+  pos_interp_kernel<<<n_total, 144, 0, st>>>(g, table, out);
   return cudaGetLastError();
 }
 

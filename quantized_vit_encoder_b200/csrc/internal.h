@@ -47,6 +47,9 @@ cudaError_t launch_quant_weight(const __nv_bfloat16* w, int N, int K, uint8_t* q
                                 cudaStream_t st);
 cudaError_t launch_rope_table(const int32_t* pos, int n, double theta, float* cs, cudaStream_t st);
 cudaError_t launch_rope_apply(__nv_bfloat16* qkv, int n, const float* cs, int v_to_f16, cudaStream_t st);
+// Bilinear interpolation of the 48 x 48 position table to each packed token's (row, col).
+cudaError_t launch_pos_interp(const GridList& g, int n_total, const __nv_bfloat16* table, __nv_bfloat16* out,
+                              cudaStream_t st);
 cudaError_t launch_positions(const GridList& g, int n_total, int32_t* pos, int32_t* cu,
                              cudaStream_t st);
 cudaError_t launch_fp8_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W, const float* sW,

@@ -79,6 +79,8 @@ _SIGS = {
     "vit_block_forward_bf16": [C.POINTER(BlockWeightsBf16), _vp, _i, _vp, _i, _i, _vp, _vp, _sz, _vp],
     "vit_merger_forward_bf16": [C.POINTER(MergerWeightsBf16), _vp, _i, _vp, _vp, _sz, _vp],
     "vitq_merger_bf16_workspace_bytes": [_i],
+    "vit_patch_embed": [_vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _vp, _sz, _vp],
+    "vitq_patch_embed_workspace_bytes": [_i],
     "vit_tower_forward_mixed": [C.POINTER(TowerWeightsMixed), _vp, _vp, _i, C.POINTER(_vp), _vp, _sz, _vp],
     "vitq_get_device_error": [_vp],
     "vitq_status_string": [_i],
@@ -90,7 +92,7 @@ _SIGS = {
     "vitq_selftest_wait_timeout": [_i, _vp],
 }
 _RES = {"vitq_block_workspace_bytes": _sz, "vitq_merger_workspace_bytes": _sz,
-        "vitq_merger_bf16_workspace_bytes": _sz,
+        "vitq_merger_bf16_workspace_bytes": _sz, "vitq_patch_embed_workspace_bytes": _sz,
         "vitq_tower_workspace_bytes": _sz, "vitq_status_string": C.c_char_p,
         "vitq_launch_count": C.c_ulonglong, "vitq_profile_start": None}
 
@@ -343,6 +345,19 @@ def tower_forward_mixed_(tower: DeviceTowerMixed, x, grids, ws, taps=None, strea
     _check(load().vit_tower_forward_mixed(C.byref(tower.struct), _p(x), C.cast(g, C.c_void_p), len(grids), tp,
                                           _p(ws), ws.numel(), _stream(stream)), "vit_tower_forward_mixed")
     return taps
+
+
+def patch_embed(pixels, grids, w, b, pos_table, out=None, ws=None, stream=None):
+    """bf16 x [n, 1152] = pixels [n, 1536] . w^T + b + interpolated position embedding."""
+    n = pixels.shape[0]
+    if out is None:
+        out = torch.empty((n, HIDDEN), dtype=torch.bfloat16, device=pixels.device)
+    if ws is None:
+        ws = workspace(int(load().vitq_patch_embed_workspace_bytes(n)), pixels.device)
+    g = (C.c_int32 * (2 * len(grids)))(*[v for hw in grids for v in hw])
+    _check(load().vit_patch_embed(_p(pixels), n, C.cast(g, C.c_void_p), len(grids), _p(w), _p(b), _p(pos_table),
+                                  _p(out), _p(ws), ws.numel(), _stream(stream)), "vit_patch_embed")
+    return out
 
 
 def block_workspace_bytes(n: int) -> int:

@@ -109,6 +109,19 @@ def merger_params(seed: int) -> dict:
     }
 
 
+PATCH_DIM, POS_GRID = 1536, 48
+
+
+def patch_params(seed: int) -> dict:
+    """bf16 patch-embedding weights [1152, 1536], bias, and the 48 x 48 position table [2304, 1152]."""
+    g = torch.Generator().manual_seed(seed)
+    return {
+        "w": _normal(g, (HIDDEN, PATCH_DIM), W_STD),
+        "b": _normal(g, (HIDDEN,), B_STD),
+        "pos": _normal(g, (POS_GRID * POS_GRID, HIDDEN), W_STD),
+    }
+
+
 def block_seed(wl: Workload, b: int) -> int:
     """Seed of block b (0-indexed) of a workload."""
     return wl.seed_base + 1 + b

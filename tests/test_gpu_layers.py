@@ -233,6 +233,25 @@ def test_mixed_tower_matches_oracle(lib):
         assert_within_drift(f64(taps[t]), ref[t], "tower_mixed_small", t)
 
 
+# ------------------------------------------------------------ patch embedding
+
+@pytest.mark.parametrize("grids", [[(16, 16)], [(36, 27)], [(1, 5), (7, 3)], [(54, 18), (46, 136), (24, 38), (32, 32)]],
+                         ids=["16x16", "36x27", "tiny", "packed4"])
+def test_patch_embed_matches_oracle(lib, grids):
+    """bf16 GEMM over the 1536 patch pixels + bias + the interpolated position embedding (a
+    single bf16 stage: the stage tolerance, and nearly every output equal to the oracle's)."""
+    from quantized_vit_encoder_b200 import vitq
+    n = sum(h * w for h, w in grids)
+    pix = wl.random_bf16((n, wl.PATCH_DIM), 90 + n, 1.0)
+    p = wl.patch_params(91)
+    got = f64(vitq.patch_embed(pix.cuda(), grids, p["w"].cuda(), p["b"].cuda(), p["pos"].cuda()))
+    assert vitq.device_error() == 0
+    ref = ov.patch_embed(f64(pix), f64(p["w"]), f64(p["b"]), f64(p["pos"]), grids)
+    assert rel_l2(got, ref) <= 1e-2
+    assert np.all(np.abs(got - ref) <= np.maximum(3e-2, bf16_ulp(ref)))
+    assert np.mean(got == ref) > 0.97
+
+
 def test_packed_tower_equals_per_image_towers(lib):
     """Block-diagonal attention and row-wise stages: each image of the packed 4-image batch
     (9164 patches) gives bitwise the same taps as that image run alone."""

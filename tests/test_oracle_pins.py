@@ -263,6 +263,55 @@ def test_bf16_gemm_exact_integer_case_and_orientation():
     assert np.array_equal(out, want)
 
 
+# ---------------------------------------------------------------- position embedding
+
+def test_pos_interp_at_table_resolution_is_the_table():
+    g = np.random.default_rng(21)
+    table = g.standard_normal((48 * 48, 5))
+    assert np.array_equal(ov.pos_embed_interp(table, 48, 48).reshape(-1, 5), table)
+
+
+def test_pos_interp_reproduces_affine_tables():
+    """Bilinear interpolation is exact on a table affine in (row, col) (and on constants)."""
+    i, j = np.meshgrid(np.arange(48.0), np.arange(48.0), indexing="ij")
+    table = np.stack([3.0 + 0.0 * i, 2.0 * i - 0.5 * j + 1.0, 0.25 * i * 1.0], -1).reshape(-1, 3)
+    for h, w in ((16, 16), (36, 27), (46, 136), (1, 7), (5, 1)):
+        out = ov.pos_embed_interp(table, h, w)
+        r = np.arange(h)[:, None] * (47.0 / (h - 1) if h > 1 else 0.0)
+        c = np.arange(w)[None, :] * (47.0 / (w - 1) if w > 1 else 0.0)
+        assert np.allclose(out[..., 0], 3.0, atol=1e-12)
+        assert np.allclose(out[..., 1], 2.0 * r - 0.5 * c + 1.0, atol=1e-10)
+        assert np.allclose(out[..., 2], 0.25 * r + 0 * c, atol=1e-10)
+
+
+def test_pos_interp_corner_points_and_midpoints():
+    """Corners take the table's corners; a grid of 95 puts every other point halfway between
+    two table rows, where the value is the mean of the two."""
+    g = np.random.default_rng(22)
+    table = g.standard_normal((48 * 48, 2))
+    T = table.reshape(48, 48, 2)
+    out = ov.pos_embed_interp(table, 95, 48)
+    assert np.allclose(out[0, 0], T[0, 0]) and np.allclose(out[-1, -1], T[-1, -1])
+    assert np.allclose(out[1], 0.5 * (T[0] + T[1]), atol=1e-12)
+    assert np.allclose(out[2], T[1], atol=1e-12)
+
+
+def test_patch_embed_adds_each_patch_its_own_position():
+    """With zero pixels and bias, x is the bf16 position embedding of each token's (row, col)
+    in token order (2x2-block order for even grids, row-major for odd)."""
+    i, j = np.meshgrid(np.arange(48.0), np.arange(48.0), indexing="ij")
+    table = np.stack([i, j], -1).reshape(-1, 2)
+    grids = [(4, 6), (3, 5)]
+    n = sum(h * w for h, w in grids)
+    x = ov.patch_embed(np.zeros((n, 8)), np.zeros((2, 8)), np.zeros(2), table, grids)
+    pos, _ = ov.packed_positions(grids)
+    want = []
+    for (h, w), start in ((grids[0], 0), (grids[1], 24)):
+        rc = pos[start:start + h * w]
+        want.append(np.stack([rc[:, 0] * 47.0 / (h - 1), rc[:, 1] * 47.0 / (w - 1)], -1))
+    assert np.array_equal(x, nm.bf16_round(np.concatenate(want)))
+
+
 # ---------------------------------------------------------------- LayerNorm / GELU
 
 def test_layernorm_moments_and_affine():
