@@ -360,6 +360,44 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     barrier()
     mixed_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
 
+    # patch embedding of the same image (pixels -> x), and a video-shaped workload:
+    # 8 frame groups of 32 x 32 patches packed through cu_seqlens (the same kernels)
+    pp = wl.patch_params(9)
+    pix = wl.random_bf16((W.n_tokens, wl.PATCH_DIM), 8, 1.0).to(dev)
+    pw, pb, ptab = pp["w"].to(dev), pp["b"].to(dev), pp["pos"].to(dev)
+    pws = vitq.workspace(int(vitq.load().vitq_patch_embed_workspace_bytes(W.n_tokens)), dev)
+    pout = torch.empty((W.n_tokens, wl.HIDDEN), dtype=torch.bfloat16, device=dev)
+    for _ in range(args.warmup):
+        vitq.patch_embed(pix, grids, pw, pb, ptab, pout, pws)
+    barrier()
+    ev0.record(stream)
+    for _ in range(nb):
+        vitq.patch_embed(pix, grids, pw, pb, ptab, pout, pws)
+    ev1.record(stream)
+    barrier()
+    patch_ms = max_over_ranks(ev0.elapsed_time(ev1) / nb)
+    vgrids = [(32, 32)] * 8
+    vn = sum(h * w for h, w in vgrids)
+    vx0 = wl.random_bf16((vn, wl.HIDDEN), 10, 1.0).to(dev)
+    vx = torch.empty_like(vx0)
+    vws = vitq.workspace(vitq.tower_workspace_bytes(vn, len(vgrids)), dev)
+    vtaps = [torch.empty((vn // 4, wl.OUT_HIDDEN), dtype=torch.bfloat16, device=dev) for _ in range(4)]
+
+    def video_step():
+        vx.copy_(vx0)
+        vitq.tower_forward_(tower, vx, vgrids, vws, vtaps)
+
+    for _ in range(2):
+        video_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        video_step()
+    ev1.record(stream)
+    barrier()
+    video_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    del vws, vx, vx0, vtaps
+
     # per-kernel device times from a profiled pass of the same step (not the timed one)
     vitq.profile_start()
     for _ in range(2):
@@ -412,6 +450,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "tower_ms": ms,
         "block_bf16_ms": block_bf16_ms,
         "mixed_tower_ms": mixed_ms,
+        "patch_embed_ms": patch_ms,
+        "video_8x32x32_tower_ms": video_ms,
         "roofline": roofline(table, peaks),
         "kernels": {k: {"launches": v["launches"] // 2, "ms_per_step": v["ms"] / 2,
                         "share": v["ms"] / sum(t["ms"] for t in table.values())} for k, v in table.items()},

@@ -252,6 +252,23 @@ def test_patch_embed_matches_oracle(lib, grids):
     assert np.mean(got == ref) > 0.97
 
 
+def test_video_frame_groups_are_independent(lib):
+    """A video as 6 frame groups of one 16 x 12 grid packed through cu_seqlens: each group's
+    taps equal that group run alone (attention never crosses a frame group)."""
+    from quantized_vit_encoder_b200 import vitq
+    grids = [(16, 12)] * 6
+    W = wl.Workload("video", tuple(grids), wl.N_BLOCKS, True, scales=(1.0,) * 6, seed_base=5300)
+    x = wl.make_input(W).cuda()
+    tower = _device_tower(W)
+    ws = vitq.workspace(vitq.tower_workspace_bytes(W.n_tokens, len(grids)))
+    packed = vitq.tower_forward_(tower, x.clone(), grids, ws)
+    for f in (0, 3, 5):
+        n0, n1 = f * 192, (f + 1) * 192
+        alone = vitq.tower_forward_(tower, x[n0:n1].clone(), [grids[f]], ws)
+        for t in range(4):
+            assert torch.equal(packed[t][n0 // 4:n1 // 4], alone[t])
+
+
 def test_packed_tower_equals_per_image_towers(lib):
     """Block-diagonal attention and row-wise stages: each image of the packed 4-image batch
     (9164 patches) gives bitwise the same taps as that image run alone."""
