@@ -73,6 +73,11 @@ constexpr int kThreads = 128 + 256 * kQTiles;
 #endif
 constexpr int kPolyEvery = VITQ_ATTN_POLY_EVERY;
 constexpr int kPolyMod = kPolyEvery > 0 ? kPolyEvery : 1;
+// 8-key group of the exponential loop after which the turn passes to the other tile (7 = at the end).
+#ifndef VITQ_ATTN_TURN_AT
+#define VITQ_ATTN_TURN_AT 5
+#endif
+constexpr int kTurnAt = VITQ_ATTN_TURN_AT;
 
 struct AttnArgs {
   const __nv_bfloat16* qkv;
@@ -390,10 +395,12 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
       }
       uint8_t* dst = pbase + r * 128 + ((c ^ (r & 7)) << 4);
       *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    if (n_q == 2 && !(x == 1 && j == n_kv - 1)) {   // hand the turn to the other tile
-      __syncwarp();
-      if (lane == 0) mbar_arrive(sm.turn(x, quad));
+      // hand the turn to the other tile a little before the end, so that its
+      // exponentials start while these finish (hides the hand-over latency)
+      if (c == kTurnAt && n_q == 2 && !(x == 1 && j == n_kv - 1)) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.turn(x, quad));
+      }
     }
     if (rescale && h == 0) {
       // O (complete up to P.V(j-1)) to the new max; done after P so the scores are dead
