@@ -464,6 +464,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tlo, const __grid_constant__ CUtensorMap thi,
                 const AttnArgs args) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  pdl_trigger();
   const int head = blockIdx.y, seq = blockIdx.z;
   const int seq_start = args.cu[seq];
   const int seq_len = args.cu[seq + 1] - seq_start;
@@ -499,6 +500,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();   // inputs may be the previous kernel's outputs
   const uint32_t tmem = *sm.tmem_holder();
   if (warp < 4) {
     if (warp == 0 && lane == 0) {
@@ -538,8 +540,7 @@ cudaError_t launch_attention(const __nv_bfloat16* qkv, int n_tokens, const int32
   if (e != cudaSuccess) return e;
   AttnArgs a{qkv, cu, out, n_tokens, scale * 1.4426950408889634f};
   dim3 grid((max_seqlen + kBM * kQTiles - 1) / (kBM * kQTiles), 16, n_seqs);
-  kern<<<grid, kThreads, kAttnSmem, st>>>(tlo, thi, a);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(kThreads), kAttnSmem, st, tlo, thi, a);
 }
 
 }  // namespace vitq

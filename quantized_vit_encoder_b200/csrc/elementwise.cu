@@ -104,6 +104,8 @@ __device__ __forceinline__ void quant_store(const float (&v)[8], bool ok, int la
 template <int ITERS>
 __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ x, int M, int K, int ldx,
                                  uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
+  pdl_trigger();
+  pdl_wait();
   const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
@@ -138,12 +140,14 @@ __global__ void __launch_bounds__(32 * kLnRows, 3)
                     const __nv_bfloat16* __restrict__ beta, int M, int K, double eps,
                     uint8_t* __restrict__ q, float* __restrict__ s, int lds, __nv_bfloat16* __restrict__ y) {
   __shared__ uint4 sg[ITERS * 32], sb[ITERS * 32];
+  pdl_trigger();
   for (int i = threadIdx.x; i < ITERS * 32; i += blockDim.x) {
     const int col = lane_col(i >> 5, i & 31);
     sg[i] = col < K ? *reinterpret_cast<const uint4*>(gamma + col) : make_uint4(0, 0, 0, 0);
     sb[i] = col < K ? *reinterpret_cast<const uint4*>(beta + col) : make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
+  pdl_wait();   // x may be the previous kernel's output
   const int row = blockIdx.x * kLnRows + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= M) return;
@@ -267,6 +271,7 @@ __global__ void __launch_bounds__(kGeluThreads, 1)
     gelu_quant_kernel(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* __restrict__ q,
                       float* __restrict__ s, int lds, __nv_bfloat16* y) {
   extern __shared__ __align__(16) uint16_t lut[];
+  pdl_trigger();
   {
     const uint4* src = reinterpret_cast<const uint4*>(g_gelu_table);
     uint4* dst = reinterpret_cast<uint4*>(lut);
@@ -274,27 +279,32 @@ __global__ void __launch_bounds__(kGeluThreads, 1)
     for (int i = 0; i < 8; ++i) dst[threadIdx.x + i * kGeluThreads] = src[threadIdx.x + i * kGeluThreads];
   }
   __syncthreads();
+  pdl_wait();
   const int steps = (K + 255) / 256;
-  const long long items = (long long)M * steps;
+  const int items = M * steps;
   const int lane = threadIdx.x & 31;
-  const long long warps = (long long)gridDim.x * (kGeluThreads / 32);
-  for (long long w = blockIdx.x * (kGeluThreads / 32) + (threadIdx.x >> 5); w < items; w += warps) {
-    const int row = (int)(w / steps);
-    const int st = (int)(w - (long long)row * steps);
+  const int warps = gridDim.x * (kGeluThreads / 32);
+  // each warp walks items w, w + warps, ...; the next item's 8 inputs per lane are
+  // loaded before the current item is processed, so the load latency overlaps the work
+  auto load = [&](int w) {
+    const int row = w / steps, col = lane_col(w - row * steps, lane);
+    return (w < items && col < K) ? *reinterpret_cast<const uint4*>(f + (size_t)row * ldf + col)
+                                  : make_uint4(0u, 0u, 0u, 0u);
+  };
+  int w = blockIdx.x * (kGeluThreads / 32) + (threadIdx.x >> 5);
+  uint4 cur = load(w);
+  for (; w < items; w += warps) {
+    const uint4 nxt = load(w + warps);
+    const int row = w / steps;
+    const int st = w - row * steps;
     const int col = lane_col(st, lane);
     const bool ok = col < K;
     float v[8];
-    if (ok) {
-      const uint4 u = *reinterpret_cast<const uint4*>(f + (size_t)row * ldf + col);
-      const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+    const uint32_t wd[4] = {cur.x, cur.y, cur.z, cur.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        v[2 * i] = __uint_as_float((uint32_t)lut[wd[i] & 0xFFFFu] << 16);
-        v[2 * i + 1] = __uint_as_float((uint32_t)lut[wd[i] >> 16] << 16);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = 0.f;
+    for (int i = 0; i < 4; ++i) {   // zero inputs (past K) read GELU(0) = 0
+      v[2 * i] = __uint_as_float((uint32_t)lut[wd[i] & 0xFFFFu] << 16);
+      v[2 * i + 1] = __uint_as_float((uint32_t)lut[wd[i] >> 16] << 16);
     }
     if (y) {   // bf16 output (may be f itself: each lane reads its 8 values before writing them)
       if (ok)
@@ -304,6 +314,7 @@ __global__ void __launch_bounds__(kGeluThreads, 1)
     } else {
       quant_store(v, ok, lane, row, col, K, q, s, lds);
     }
+    cur = nxt;
   }
 }
 
@@ -312,6 +323,8 @@ __global__ void __launch_bounds__(kGeluThreads, 1)
 
 __global__ void quant_weight_kernel(const __nv_bfloat16* __restrict__ w, int N, int K,
                                     uint8_t* __restrict__ q, float* __restrict__ s) {
+  pdl_trigger();
+  pdl_wait();
   const int nb = blockIdx.y, kb = blockIdx.x;
   const int nkb = gridDim.x;
   const int t = threadIdx.x;
@@ -356,6 +369,8 @@ __global__ void quant_weight_kernel(const __nv_bfloat16* __restrict__ w, int N, 
 
 __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int n, double theta,
                                   float* __restrict__ cs) {
+  pdl_trigger();
+  pdl_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= n * 36) return;
   const int t = idx / 36, j = idx - t * 36;
@@ -377,6 +392,8 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int n, double
 // writes after it, so the in-place update never reads a rotated value.
 __global__ void __launch_bounds__(432) rope_apply_kernel(__nv_bfloat16* __restrict__ qkv,
                                                          const float* __restrict__ cs, int v_to_f16) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   const int c = threadIdx.x;
   __nv_bfloat16* base = qkv + (size_t)t * 3456;
@@ -467,6 +484,8 @@ constexpr int kPosGrid = 48;
 
 __global__ void __launch_bounds__(144) pos_interp_kernel(GridList grids, const __nv_bfloat16* __restrict__ table,
                                                          __nv_bfloat16* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x;
   int img, r, c;
   token_place(grids, t, img, r, c);
@@ -496,6 +515,8 @@ __global__ void __launch_bounds__(144) pos_interp_kernel(GridList grids, const _
 
 __global__ void positions_kernel(GridList grids, int n_total, int32_t* __restrict__ pos,
                                  int32_t* __restrict__ cu) {
+  pdl_trigger();
+  pdl_wait();
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
   if (t == 0) {
     int acc = 0;
@@ -542,8 +563,8 @@ template <int IT>
 static void qa_launch(const __nv_bfloat16* x, int M, int K, int ldx, uint8_t* q, float* s, int lds,
                       cudaStream_t st) {
   const int threads = 128;
-  quant_act_kernel<IT><<<(unsigned)(((long long)M * 32 + threads - 1) / threads), threads, 0, st>>>(
-      x, M, K, ldx, q, s, lds);
+  launch_pdl(quant_act_kernel<IT>, dim3((unsigned)(((long long)M * 32 + threads - 1) / threads)), dim3(threads), 0,
+             st, x, M, K, ldx, q, s, lds);
 }
 
 cudaError_t launch_quant_act(const __nv_bfloat16* x, int M, int K, int ldx, uint8_t* q, float* s,
@@ -567,11 +588,11 @@ static void ln_launch(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* g,
                       const __nv_bfloat16* b, int M, int K, double eps, uint8_t* q, float* s, int lds,
                       __nv_bfloat16* y, cudaStream_t st) {
   if (y)
-    ln_quant_kernel<IT, true><<<(unsigned)((M + kLnRows - 1) / kLnRows), 32 * kLnRows, 0, st>>>(
-        x, ldx, g, b, M, K, eps, q, s, lds, y);
+    launch_pdl(ln_quant_kernel<IT, true>, dim3((unsigned)((M + kLnRows - 1) / kLnRows)), dim3(32 * kLnRows), 0, st,
+               x, ldx, g, b, M, K, eps, q, s, lds, y);
   else
-    ln_quant_kernel<IT, false><<<(unsigned)((M + kLnRows - 1) / kLnRows), 32 * kLnRows, 0, st>>>(
-        x, ldx, g, b, M, K, eps, q, s, lds, y);
+    launch_pdl(ln_quant_kernel<IT, false>, dim3((unsigned)((M + kLnRows - 1) / kLnRows)), dim3(32 * kLnRows), 0, st,
+               x, ldx, g, b, M, K, eps, q, s, lds, y);
 }
 
 cudaError_t launch_ln(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,
@@ -605,37 +626,37 @@ cudaError_t launch_gelu(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* 
   if (e != cudaSuccess) return e;
   const long long warps = (long long)M * ((K + 255) / 256);
   const long long ctas = (warps + kGeluThreads / 32 - 1) / (kGeluThreads / 32);
-  gelu_quant_kernel<<<(unsigned)(ctas < num_sms ? ctas : num_sms), kGeluThreads, kGeluSmem, st>>>(
+  return launch_pdl(gelu_quant_kernel, dim3((unsigned)(ctas < num_sms ? ctas : num_sms)), dim3(kGeluThreads),
+                    kGeluSmem, st,
       f, M, K, ldf, q, s, lds, y);
-  return cudaGetLastError();
 }
 
 cudaError_t launch_quant_weight(const __nv_bfloat16* w, int N, int K, uint8_t* q, float* s,
                                 cudaStream_t st) {
   if (N == 0 || K == 0) return cudaSuccess;
   dim3 grid((K + 127) / 128, (N + 127) / 128);
-  quant_weight_kernel<<<grid, 256, 0, st>>>(w, N, K, q, s);
+  launch_pdl(quant_weight_kernel, grid, dim3(256), 0, st, w, N, K, q, s);
   return cudaGetLastError();
 }
 
 cudaError_t launch_rope_table(const int32_t* pos, int n, double theta, float* cs, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const int threads = 256;
-  rope_table_kernel<<<(unsigned)(((long long)n * 36 + threads - 1) / threads), threads, 0, st>>>(
+  launch_pdl(rope_table_kernel, dim3((unsigned)(((long long)n * 36 + threads - 1) / threads)), dim3(threads), 0, st,
       pos, n, theta, cs);
   return cudaGetLastError();
 }
 
 cudaError_t launch_rope_apply(__nv_bfloat16* qkv, int n, const float* cs, int v_to_f16, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
-  rope_apply_kernel<<<n, 432, 0, st>>>(qkv, cs, v_to_f16);
+  launch_pdl(rope_apply_kernel, dim3(n), dim3(432), 0, st, qkv, cs, v_to_f16);
   return cudaGetLastError();
 }
 
 cudaError_t launch_pos_interp(const GridList& g, int n_total, const __nv_bfloat16* table, __nv_bfloat16* out,
                               cudaStream_t st) {
   if (n_total == 0) return cudaSuccess;
-  pos_interp_kernel<<<n_total, 144, 0, st>>>(g, table, out);
+  launch_pdl(pos_interp_kernel, dim3(n_total), dim3(144), 0, st, g, table, out);
   return cudaGetLastError();
 }
 
@@ -643,7 +664,7 @@ cudaError_t launch_positions(const GridList& g, int n_total, int32_t* pos, int32
                              cudaStream_t st) {
   const int threads = 256;
   const int blocks = n_total > 0 ? (n_total + threads - 1) / threads : 1;
-  positions_kernel<<<blocks, threads, 0, st>>>(g, n_total, pos, cu);
+  launch_pdl(positions_kernel, dim3(blocks), dim3(threads), 0, st, g, n_total, pos, cu);
   return cudaGetLastError();
 }
 

@@ -228,6 +228,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BN>::THREADS, 1)
                      const Bf16Args args) {
   using Cfg = Bf16Cfg<BN>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  pdl_trigger();
   Bf16Smem<BN> sm;
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -255,6 +256,7 @@ __global__ void __launch_bounds__(Bf16Cfg<BN>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();   // inputs may be the previous kernel's outputs
   const uint32_t tmem_base = *sm.tmem_holder();
   if (warp < Cfg::EPI_WARP0) {
     if (warp == 0 && lane == 0) {
@@ -286,8 +288,7 @@ cudaError_t bf16_launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const
   if (e != cudaSuccess) return e;
   const int tiles = ((a.M + Cfg::BM - 1) / Cfg::BM) * ((a.N + BN - 1) / BN);
   const int grid = tiles < num_sms ? tiles : num_sms;
-  bf16_gemm_kernel<BN><<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(tmA, tmB, tmC, tmR, a);
-  return cudaGetLastError();
+  return launch_pdl(bf16_gemm_kernel<BN>, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, tmC, tmR, a);
 }
 
 }  // namespace

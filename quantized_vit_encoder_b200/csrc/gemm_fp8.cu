@@ -371,6 +371,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kPair>::THREADS, 1)
                     const GemmArgs args) {
   using Cfg = GemmCfg<BN, kPair>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  pdl_trigger();
   GemmSmem<BN, kPair> sm;
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -409,6 +410,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kPair>::THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  pdl_wait();   // inputs may be the previous kernel's outputs
   const uint32_t tmem_base = *sm.tmem_holder();
 
   if (warp < Cfg::EPI_WARP0) {
@@ -459,8 +461,7 @@ cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUte
   const int tiles = ((a.M + Cfg::TILE_M - 1) / Cfg::TILE_M) * ((a.N + BN - 1) / BN);
   if (!kPair) {
     const int grid = tiles < num_sms ? tiles : num_sms;
-    kern<<<grid, Cfg::THREADS, Cfg::SMEM, st>>>(tmA, tmB, tmC, tmR, a);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(Cfg::THREADS), Cfg::SMEM, st, tmA, tmB, tmC, tmR, a);
   }
   const int pairs = tiles < num_sms / 2 ? tiles : num_sms / 2;
   cudaLaunchConfig_t cfg = {};
@@ -468,13 +469,15 @@ cudaError_t launch_bn(const CUtensorMap& tmA, const CUtensorMap& tmB, const CUte
   cfg.blockDim = dim3(Cfg::THREADS, 1, 1);
   cfg.dynamicSmemBytes = Cfg::SMEM;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl_enabled() ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, tmA, tmB, tmC, tmR, a);
 }
 

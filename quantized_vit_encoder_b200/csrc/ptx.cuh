@@ -147,6 +147,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* tm,
       : "memory");
 }
 
+// --------------------------------------------------- programmatic dependent launch
+// Kernels are launched so that the next kernel on the stream may be scheduled
+// while this one drains (pdl_trigger, at the start: the dependent grid is only
+// scheduled once every CTA of this grid has issued it, i.e. is resident), and
+// each kernel waits for its predecessor to complete, with its writes visible,
+// before touching global memory the predecessor may read or write (pdl_wait).
+// Without a programmatic predecessor pdl_wait returns at once.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ CTA pairs
 // A cluster of two CTAs sharing one tcgen05 MMA (cta_group::2): the leader
 // (rank 0) issues the MMAs, which read operands from both CTAs' shared memory
