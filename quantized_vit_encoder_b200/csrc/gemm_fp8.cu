@@ -33,7 +33,8 @@
 namespace vitq {
 namespace {
 
-// BN = 128: 6 warps (TMA, MMA, 4 epilogue warps).  BN = 256: 12 warps
+// BN = 128: 10 warps (TMA, MMA, 8 epilogue warps, one per 64 columns x 32 rows).
+// BN = 256: 12 warps
 // (warpgroup 0 = TMA, MMA and two idle warps, which give registers away with
 // setmaxnreg; warpgroups 1-2 = 8 epilogue warps, one per 128 columns x 32 rows).
 template <int BN, bool kPair = false>
@@ -46,14 +47,18 @@ struct GemmCfg {
   static constexpr int B_BYTES = B_ROWS * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NBUF = 512 / BN;
-  static constexpr int EPI_WARPS = BN / 32;
+  // columns per epilogue warp: 64 for BN = 128 (8 epilogue warps: one TMEM round
+  // trip per K block each), 128 for BN = 256 (the register file holds no more)
+  static constexpr int COLS = BN == 128 ? 64 : 128;
+  static constexpr int NH = COLS / 64;                // 64-column halves per warp
+  static constexpr int EPI_WARPS = (BN / COLS) * 4;
   static constexpr int TEMPTY_COUNT = EPI_WARPS * (kPair ? 2 : 1);   // both CTAs' epilogues free a buffer
   static constexpr int EPI_WARP0 = BN == 256 ? 4 : 2;
-  static constexpr int THREADS = BN == 256 ? 384 : 192;
+  static constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
   static constexpr bool SPLIT_REGS = BN == 256;
   static constexpr int MIN_LAUNCH_REGS = 168;   // 384 x 168 >= 128 x 56 + 256 x 224 (BN = 256)
-  static constexpr int OUT_WARP_BYTES = 2 * 4096;   // two 64-column SW128 boxes of 32 rows
-  static constexpr int OUT_BYTES = EPI_WARPS * (OUT_WARP_BYTES + 256);   // + the warp's 128 bias values
+  static constexpr int OUT_WARP_BYTES = NH * 4096;  // 64-column SW128 boxes of 32 rows
+  static constexpr int OUT_BYTES = EPI_WARPS * (OUT_WARP_BYTES + COLS * 2);   // + the warp's bias values
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF + EPI_WARPS) * 8 + 16;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + OUT_BYTES + 1024 + BAR_BYTES;
 };
@@ -81,7 +86,8 @@ struct GemmSmem {
     return base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + (size_t)w * Cfg::OUT_WARP_BYTES;
   }
   __device__ uint8_t* bias(int w) const {
-    return base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + (size_t)Cfg::EPI_WARPS * Cfg::OUT_WARP_BYTES + w * 256;
+    return base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + (size_t)Cfg::EPI_WARPS * Cfg::OUT_WARP_BYTES +
+           w * Cfg::COLS * 2;
   }
   __device__ uint64_t* bars() const {
     return reinterpret_cast<uint64_t*>(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES);
@@ -215,9 +221,9 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;                         // TMEM lane quadrant this warp may access
   const int ew = warp - Cfg::EPI_WARP0;              // epilogue warp index
-  const int cg = ew >> 2;                            // which 128-column group of the tile
+  const int cg = ew >> 2;                            // which COLS-column group of the tile
   const int r_in = quad * 32 + lane;
-  uint8_t* stg = sm.out(ew);                         // staging: [2 boxes][32 rows][128 B], SW128
+  uint8_t* stg = sm.out(ew);                         // staging: [NH boxes][32 rows][128 B], SW128
   const uint32_t stg_u32 = smem_u32(stg);
   const bool has_res = g.residual != nullptr;
   // the leader's tempty barriers count both CTAs' epilogue warps
@@ -229,30 +235,31 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
     const int m0 = mt * Cfg::TILE_M + rank * Cfg::BM;
     const int n0 = nt * BN;
     const int row = m0 + r_in;
-    const int col0 = n0 + cg * 128;
+    const int col0 = n0 + cg * Cfg::COLS;
     const int y0 = m0 + quad * 32;                   // first row of this warp's staging tile
     const bool row_ok = row < g.M;
     const bool col_ok = col0 < g.N;
-    // this warp's 128 bias values (lane l: columns 4l..4l+3), loaded now and
+    // this warp's COLS bias values (lane l: columns 4l..4l+3), loaded now and
     // parked in shared memory after the K loop
     uint2 bias_l = make_uint2(0u, 0u);
-    if (g.bias && col0 + 4 * lane < g.N) bias_l = __ldg(reinterpret_cast<const uint2*>(g.bias + col0 + 4 * lane));
+    if (g.bias && 4 * lane < Cfg::COLS && col0 + 4 * lane < g.N)
+      bias_l = __ldg(reinterpret_cast<const uint2*>(g.bias + col0 + 4 * lane));
     // the residual tile is requested at the start of the tile, once the previous
     // tile's stores have read the staging tile
     if (has_res) {
       if (lane == 0) {
         bulk_wait_read_all();
         mbar_arrive_expect_tx(sm.res_full(ew), Cfg::OUT_WARP_BYTES);
-        tma_load_2d(stg_u32, tmR, col0, y0, sm.res_full(ew));
-        tma_load_2d(stg_u32 + 4096, tmR, col0 + 64, y0, sm.res_full(ew));
+#pragma unroll
+        for (int h = 0; h < Cfg::NH; ++h) tma_load_2d(stg_u32 + h * 4096, tmR, col0 + h * 64, y0, sm.res_full(ew));
       }
       __syncwarp();
     }
     const float* sa_ptr = g.sA + row;
     const float* sw_ptr = g.sW + (size_t)(col0 >> 7) * nkb;
-    uint64_t acc[64];
+    uint64_t acc[Cfg::NH * 32];
 #pragma unroll
-    for (int j = 0; j < 64; ++j) acc[j] = 0ull;
+    for (int j = 0; j < Cfg::NH * 32; ++j) acc[j] = 0ull;
     // scales are loaded one K block ahead so their latency hides behind the previous block
     float sa_next = row_ok ? __ldg(sa_ptr) : 0.f;
     float sw_next = col_ok ? __ldg(sw_ptr) : 0.f;
@@ -270,9 +277,9 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
       if (!__all_sync(0xffffffffu, ok)) return;
       if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(5, cnt);  // epilogue: partial ready
       tc_fence_after();
-      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + cg * 128;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + cg * Cfg::COLS;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
+      for (int h = 0; h < Cfg::NH; ++h) {
         uint32_t r0[32], r1[32];
         tmem_ld32(taddr + h * 64, r0);
         tmem_ld32(taddr + h * 64 + 32, r1);
@@ -297,7 +304,7 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
     }
     if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(7, it);  // epilogue: K loop done
     uint8_t* bias_s = sm.bias(ew);
-    *reinterpret_cast<uint2*>(bias_s + lane * 8) = bias_l;
+    if (4 * lane < Cfg::COLS) *reinterpret_cast<uint2*>(bias_s + lane * 8) = bias_l;
     if (has_res) {
       const bool ok = mbar_wait(sm.res_full(ew), it & 1u, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
@@ -309,7 +316,7 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
     // bias + residual, bf16, into the staging tile (row = lane, 16-byte chunk c of
     // box h at position c ^ (lane & 7))
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < Cfg::NH; ++h) {
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const int c8 = h * 8 + c;
@@ -355,8 +362,9 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
     if (lane == 0) {
       // TMA clips rows >= M and columns >= N; boxes wholly outside are skipped
       if (y0 < g.M) {
-        if (col0 < g.N) tma_store_2d(tmC, stg_u32, col0, y0);
-        if (col0 + 64 < g.N) tma_store_2d(tmC, stg_u32 + 4096, col0 + 64, y0);
+#pragma unroll
+        for (int h = 0; h < Cfg::NH; ++h)
+          if (col0 + h * 64 < g.N) tma_store_2d(tmC, stg_u32 + h * 4096, col0 + h * 64, y0);
       }
       bulk_commit_group();
     }
