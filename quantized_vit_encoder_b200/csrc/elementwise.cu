@@ -20,42 +20,88 @@ namespace {
 
 constexpr float kE4M3Max = 448.0f;
 
-// The quotient y / s that decides an E4M3 code.  The code depends only on which
-// side of an E4M3 rounding midpoint fl(y / s) lies; y * fl(1 / s) is within a
-// few ulps of fl(y / s), so the exact IEEE division is taken only when that
-// product lies within 16 ulps of a midpoint (mantissa tail 0x80000) or below
-// the normal E4M3 range.  The result therefore always encodes like fl(y / s).
-__device__ __forceinline__ float e4m3_quotient(float y, float s, float r) {
-  float q = y * r;
-  const uint32_t b = __float_as_uint(q) & 0x7FFFFFFFu;
-  // mantissa tail within 16 of 0x80000  <=>  ((b - 0x7FFF0) mod 2^20) <= 32
-  if (b < 0x3C800000u || ((b - 0x7FFF0u) & 0xFFFFFu) <= 32u) q = __fdiv_rn(y, s);
-  return q;
+// Two fp32 values (packed) -> bf16x2, round to nearest even (lo in bits 0..15).
+__device__ __forceinline__ uint32_t bf16x2_of(uint64_t v) {
+  const float2 f = f2unpack(v);
+  uint32_t w;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(f.y), "f"(f.x));
+  return w;
+}
+// ------------------------------------------------ exact block-128 quantisation
+// Group scale fl32(amax / 448) without a division: q0 = fl(amax * R) with
+// R = fl(1/448), then one FMA correction.  For every bf16 amax from 2^-100 to
+// the largest finite bf16 this equals the IEEE quotient (checked exhaustively);
+// every amax here is a bf16 value (the quantised inputs are bf16).  Other
+// values take the IEEE division.
+__device__ __forceinline__ float e4m3_scale(float amax) {
+  if (amax >= 7.88860905e-31f && amax <= 3.38953139e38f) {
+    constexpr float R = 1.0f / 448.0f;
+    const float q0 = __fmul_rn(amax, R);
+    return __fmaf_rn(__fmaf_rn(-q0, kE4M3Max, amax), R, q0);
+  }
+  return __fdiv_rn(amax, kE4M3Max);
 }
 
-// Quantise 8 consecutive values of one 128-column group given the group scale.
+// E4M3 codes of 8 values of one group, equal to code(fl32(y / s)) without a
+// division.  r = rcp.approx(s) is within 1 ulp of 1/s, so rl = r - 64 ulps
+// <= 1/s <= r + 64 ulps = rh.  For y >= 0, y rl <= y / s <= y rh, and rounding
+// to fp32 and then to E4M3 is monotone, so code(fl(y rl)) <= code(fl(y / s))
+// <= code(fl(y rh)) (mirrored for y < 0): where the outer codes agree, they are
+// the answer.  A pair where they differ (about 2^-12 of pairs) divides exactly.
 // A scale below the fp32 normal range (amax < 448 * 2^-126) has no finite
 // reciprocal; those groups always divide exactly.
 __device__ __forceinline__ uint2 quant8(const float (&v)[8], float s) {
-  uint32_t c[4] = {0u, 0u, 0u, 0u};
-  if (s >= 1.17549435e-38f) {
-    const float r = __frcp_rn(s);
+  uint32_t w[2] = {0u, 0u};
+  if (s >= 1.17549435e-38f && s <= 1e36f) {   // normal, with a normal reciprocal
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
+    const uint32_t rb = __float_as_uint(r);
+    const uint64_t rl = f2pack(__uint_as_float(rb - 64u), __uint_as_float(rb - 64u));
+    const uint64_t rh = f2pack(__uint_as_float(rb + 64u), __uint_as_float(rb + 64u));
+    uint32_t lo[4], hi[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      c[i] = cvt_e4m3x2(e4m3_quotient(v[2 * i], s, r), e4m3_quotient(v[2 * i + 1], s, r));
+    for (int i = 0; i < 4; ++i) {
+      const uint64_t x = f2pack(v[2 * i], v[2 * i + 1]);
+      const float2 a = f2unpack(fmul2(x, rl)), b = f2unpack(fmul2(x, rh));
+      lo[i] = cvt_e4m3x2(a.x, a.y);
+      hi[i] = cvt_e4m3x2(b.x, b.y);
+    }
+    w[0] = __byte_perm(lo[0], lo[1], 0x5410);
+    w[1] = __byte_perm(lo[2], lo[3], 0x5410);
+    const uint32_t h0 = __byte_perm(hi[0], hi[1], 0x5410), h1 = __byte_perm(hi[2], hi[3], 0x5410);
+    if ((w[0] != h0) | (w[1] != h1)) {   // rare: a pair straddles an E4M3 rounding boundary
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (lo[i] != hi[i]) lo[i] = cvt_e4m3x2(__fdiv_rn(v[2 * i], s), __fdiv_rn(v[2 * i + 1], s));
+      }
+      w[0] = __byte_perm(lo[0], lo[1], 0x5410);
+      w[1] = __byte_perm(lo[2], lo[3], 0x5410);
+    }
   } else if (s > 0.f) {
+    uint32_t c[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      c[i] = cvt_e4m3x2(__fdiv_rn(v[2 * i], s), __fdiv_rn(v[2 * i + 1], s));
+    for (int i = 0; i < 4; ++i) c[i] = cvt_e4m3x2(__fdiv_rn(v[2 * i], s), __fdiv_rn(v[2 * i + 1], s));
+    w[0] = __byte_perm(c[0], c[1], 0x5410);
+    w[1] = __byte_perm(c[2], c[3], 0x5410);
   }
-  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+  return make_uint2(w[0], w[1]);
 }
 
-// Max over the 16 lanes of a half warp.
-__device__ __forceinline__ float half_warp_max(float v) {
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
+// Max of |v| over 8 values (NaN ignored, like fmaxf).
+__device__ __forceinline__ float amax8(const float (&v)[8]) {
+  const float a = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
+                        fmaxf(fabsf(v[6]), fabsf(v[7])));
+  return a == a ? a : 0.f;
+}
+
+// Max over each half warp of non-negative values: lanes 0-15 get the max of
+// lanes 0-15, lanes 16-31 that of lanes 16-31 (non-negative floats order like
+// their bit patterns).  All 32 lanes must take part.
+__device__ __forceinline__ float half_warp_max(float a, int lane) {
+  const uint32_t u = __float_as_uint(a);
+  const uint32_t m0 = __reduce_max_sync(0xffffffffu, lane < 16 ? u : 0u);
+  const uint32_t m1 = __reduce_max_sync(0xffffffffu, lane < 16 ? 0u : u);
+  return __uint_as_float(lane < 16 ? m0 : m1);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
@@ -71,27 +117,15 @@ __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float (&v)[8]
   unpack8(*reinterpret_cast<const uint4*>(p), v);
 }
 
-// Exact value of a bf16 bit pattern as fp64, by moving its fields (zero and
-// bf16 subnormals, below 1.2e-38, give 0).
-__device__ __forceinline__ double bf16_bits_to_f64(uint32_t h) {
-  const uint32_t e = (h >> 7) & 0xFFu;
-  uint64_t bits = (uint64_t)(h & 0x8000u) << 48;
-  if (e) bits |= ((uint64_t)(e + 896u) << 52) | ((uint64_t)(h & 0x7Fu) << 45);
-  return __longlong_as_double((long long)bits);
-}
-
 // Lane layout shared by the row kernels: a warp covers 256 columns per step;
 // lanes 0-15 hold group 2*step, lanes 16-31 group 2*step+1, 8 columns each.
 __device__ __forceinline__ int lane_col(int step, int lane) { return step * 256 + lane * 8; }
 
-// Group amax over the half warp, scale, codes and scale store for one step.
+// Group amax over the half warp, scale, codes and scale store for one step
+// (lane layout of lane_col; all 32 lanes take part).
 __device__ __forceinline__ void quant_store(const float (&v)[8], bool ok, int lane, int row, int col, int K,
                                             uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
-  float a = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(v[i]));
-  a = half_warp_max(a);
-  const float sc = __fdiv_rn(a, kE4M3Max);
+  const float sc = e4m3_scale(half_warp_max(amax8(v), lane));
   if (ok) {
     *reinterpret_cast<uint2*>(q + (size_t)row * K + col) = quant8(v, sc);
     if ((lane & 15) == 0) s[(size_t)(col >> 7) * lds + row] = sc;
@@ -125,52 +159,61 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ x, int M, int
 }
 
 // --------------------------------------------------------- LayerNorm + quant
-// One warp per row, eight rows per CTA; gamma and beta are staged once per CTA
-// in shared memory.  The statistics are exact fp64 sums of the bf16 inputs
-// (sum and sum of squares); the normalised value is evaluated in fp32 and,
-// when it lies within its error bound of a bf16 rounding midpoint, recomputed
-// in fp64, so the bf16 result is the rounding of the fp64 value
-// (x - mean) * rstd * gamma + beta.
+// A half warp per row (lane l of the half holds columns 128c + 8l, so each
+// 128-column group is one chunk c across the half warp), eight rows per CTA;
+// gamma and beta are staged once per CTA in shared memory.  The
+// statistics are exact fp64 sums of the bf16 inputs (sum and sum of squares).
+// The normalised value y = (x - mean) rstd gamma + beta is evaluated in fp32;
+// its error is below (|y| + 2|beta|) 2^-20 + 2^-126, and where y minus and
+// plus that bound round to the same bf16 value, that value is the rounding of
+// the exact y.  Elsewhere (about 2^-11 of the pairs) y is recomputed in fp64.
+
+// bf16 pair of ((x - mean) rstd gamma + beta) evaluated in fp64.
+__device__ __noinline__ uint32_t ln_pair_fp64(float x0, float x1, float g0, float g1, float b0, float b1,
+                                              double mean, double rstd) {
+  const __nv_bfloat16 h0 = __double2bfloat16(((double)x0 - mean) * rstd * (double)g0 + (double)b0);
+  const __nv_bfloat16 h1 = __double2bfloat16(((double)x1 - mean) * rstd * (double)g1 + (double)b1);
+  return (uint32_t)*reinterpret_cast<const uint16_t*>(&h0) | ((uint32_t)*reinterpret_cast<const uint16_t*>(&h1) << 16);
+}
 
 constexpr int kLnRows = 8;
 
+constexpr int kLnMaxChunks = 36;   // K <= 4608
+
+// ITERS = chunks per row (1..9, unrolled), or 0: wider rows, chunk count from K.
 template <int ITERS, bool kOutBf16>
-__global__ void __launch_bounds__(32 * kLnRows, 3)
+__global__ void __launch_bounds__(16 * kLnRows, 6)
     ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx, const __nv_bfloat16* __restrict__ gamma,
                     const __nv_bfloat16* __restrict__ beta, int M, int K, double eps,
                     uint8_t* __restrict__ q, float* __restrict__ s, int lds, __nv_bfloat16* __restrict__ y) {
-  __shared__ uint4 sg[ITERS * 32], sb[ITERS * 32];
+  constexpr int kSm = ITERS > 0 ? ITERS : kLnMaxChunks;
+  __shared__ uint4 sg[kSm * 16], sb[kSm * 16];
+  const int nch = ITERS > 0 ? ITERS : (K + 127) >> 7;
   pdl_trigger();
-  for (int i = threadIdx.x; i < ITERS * 32; i += blockDim.x) {
-    const int col = lane_col(i >> 5, i & 31);
+  for (int i = threadIdx.x; i < nch * 16; i += blockDim.x) {
+    const int col = i * 8;
     sg[i] = col < K ? *reinterpret_cast<const uint4*>(gamma + col) : make_uint4(0, 0, 0, 0);
     sb[i] = col < K ? *reinterpret_cast<const uint4*>(beta + col) : make_uint4(0, 0, 0, 0);
   }
   __syncthreads();
   pdl_wait();   // x may be the previous kernel's output
-  const int row = blockIdx.x * kLnRows + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= M) return;
-  // Rows of up to 8 steps stay in registers; wider rows (the merger's 4608) are
-  // read again from L1/L2 in the second pass.
-  constexpr bool kKeep = ITERS <= 8;
-  constexpr int kHeld = kKeep ? ITERS : 1;
-  const __nv_bfloat16* xr = x + (size_t)row * ldx;
-  auto load_step = [&](int it) {
-    const int col = lane_col(it, lane);
-    return col < K ? *reinterpret_cast<const uint4*>(xr + col) : make_uint4(0, 0, 0, 0);
+  const int lane = threadIdx.x & 31, l = lane & 15;
+  const int row = blockIdx.x * kLnRows + (threadIdx.x >> 4);
+  // both halves of a warp stay to the end (the group max is a full-warp reduction)
+  if (blockIdx.x * kLnRows + ((threadIdx.x >> 5) << 1) >= M) return;
+  const bool row_ok = row < M;
+  const __nv_bfloat16* xr = x + (size_t)(row_ok ? row : 0) * ldx;
+  // the second pass reads the row again (from L1, where the first pass left it)
+  auto load_chunk = [&](int c) {
+    const int col = c * 128 + l * 8;
+    return (row_ok && col < K) ? *reinterpret_cast<const uint4*>(xr + col) : make_uint4(0, 0, 0, 0);
   };
-  uint4 raw[kHeld];
-  if (kKeep) {
-#pragma unroll
-    for (int it = 0; it < kHeld; ++it) raw[it] = load_step(it);
-  }
   // exact fp64 sums of the bf16 inputs (bf16 -> fp32 -> fp64 is exact); 2 chains each
   double s1[2] = {0.0, 0.0}, s2[2] = {0.0, 0.0};
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
+  for (int c = 0; c < nch; ++c) {
     float v[8];
-    unpack8(kKeep ? raw[kKeep ? it : 0] : load_step(it), v);
+    unpack8(load_chunk(c), v);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const double d = (double)v[i];
@@ -180,7 +223,7 @@ __global__ void __launch_bounds__(32 * kLnRows, 3)
   }
   double t1 = s1[0] + s1[1], t2 = s2[0] + s2[1];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
+  for (int o = 8; o > 0; o >>= 1) {
     t1 += __shfl_xor_sync(0xffffffffu, t1, o);
     t2 += __shfl_xor_sync(0xffffffffu, t2, o);
   }
@@ -188,56 +231,45 @@ __global__ void __launch_bounds__(32 * kLnRows, 3)
   const double var = fmax(t2 / (double)K - mean * mean, 0.0);
   const double rstd = 1.0 / sqrt(var + eps);
   const float mh = (float)mean, ml = (float)(mean - (double)mh), r32 = (float)rstd;
+  const uint64_t nmh = f2pack(-mh, -mh), nml = f2pack(-ml, -ml), rr = f2pack(r32, r32);
 #pragma unroll
-  for (int it = 0; it < ITERS; ++it) {
-    const int col = lane_col(it, lane);
-    const bool ok = col < K;
-    const uint4 rv = kKeep ? raw[kKeep ? it : 0] : load_step(it);
-    float v[8];
-    unpack8(rv, v);
-    if (ok) {
-      float g[8], b[8];
-      unpack8(sg[it * 32 + lane], g);
-      unpack8(sb[it * 32 + lane], b);
-      bool slow = false;
+  for (int c = 0; c < nch; ++c) {
+    const int col = c * 128 + l * 8;
+    const bool ok = row_ok && col < K;
+    float v[8], g[8], b[8];
+    unpack8(load_chunk(c), v);
+    unpack8(sg[c * 16 + l], g);
+    unpack8(sb[c * 16 + l], b);
+    uint32_t w[4];
+    uint32_t slow = 0u;   // pairs whose bracket straddles a bf16 rounding boundary
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float t = ((v[i] - mh) - ml) * r32;
-        const float y = fmaf(t, g[i], b[i]);
-        // fp32 error of y is below (|t g| + |b|) 2^-20; distance of y to the nearest
-        // bf16 rounding midpoint = half a bf16 ulp (from y's exponent) - |y - bf16(y)|
-        const float yr = __bfloat162float(__float2bfloat16_rn(y));
-        const float half = __uint_as_float((__float_as_uint(y) & 0x7F800000u) - (8u << 23));
-        const float err = (fabsf(t * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;
-        slow |= (half - fabsf(y - yr) <= err) | (fabsf(y) < 1e-30f);
-        v[i] = yr;
-      }
-      if (slow) {   // rare: redo the flagged values in fp64 from the inputs
-        float xi[8];
-        unpack8(rv, xi);
-        unpack8(sg[it * 32 + lane], g);
-        unpack8(sb[it * 32 + lane], b);
-#pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
-          const float t = ((xi[i] - mh) - ml) * r32;
-          const float y = fmaf(t, g[i], b[i]);
-          const float yr = __bfloat162float(__float2bfloat16_rn(y));
-          const float half = __uint_as_float((__float_as_uint(y) & 0x7F800000u) - (8u << 23));
-          const float err = (fabsf(t * g[i]) + fabsf(b[i])) * 9.5367431640625e-07f;
-          if (half - fabsf(y - yr) <= err || fabsf(y) < 1e-30f) {
-            const double yd = ((double)xi[i] - mean) * rstd * (double)g[i] + (double)b[i];
-            v[i] = __bfloat162float(__double2bfloat16(yd));
-          }
-        }
-      }
+    for (int i = 0; i < 4; ++i) {
+      const uint64_t t = fmul2(fadd2(fadd2(f2pack(v[2 * i], v[2 * i + 1]), nmh), nml), rr);
+      const uint64_t yy = ffma2(t, f2pack(g[2 * i], g[2 * i + 1]), f2pack(b[2 * i], b[2 * i + 1]));
+      const float2 yf = f2unpack(yy);
+      const float e0 = fmaf(fabsf(yf.x), 0x1p-20f, fmaf(fabsf(b[2 * i]), 0x1p-19f, 0x1p-126f));
+      const float e1 = fmaf(fabsf(yf.y), 0x1p-20f, fmaf(fabsf(b[2 * i + 1]), 0x1p-19f, 0x1p-126f));
+      const uint64_t e = f2pack(e0, e1);
+      const uint32_t lo = bf16x2_of(ffma2(e, f2pack(-1.f, -1.f), yy)), hi = bf16x2_of(fadd2(yy, e));
+      slow |= (uint32_t)(lo != hi) << i;
+      w[i] = lo;
     }
-    if (kOutBf16) {   // bf16 output (the bf16 blocks and mergers): values are already bf16
-      if (ok)
-        *reinterpret_cast<uint4*>(y + (size_t)row * K + col) =
-            make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                       pack_bf16x2(v[6], v[7]));
+    if (slow) {   // rare (about 2^-11 of the pairs): those pairs in fp64
+#pragma unroll 1
+      for (int i = 0; i < 4; ++i)
+        if ((slow >> i) & 1u)
+          w[i] = ln_pair_fp64(v[2 * i], v[2 * i + 1], g[2 * i], g[2 * i + 1], b[2 * i], b[2 * i + 1], mean, rstd);
+    }
+    if (kOutBf16) {   // bf16 output (the bf16 blocks and mergers)
+      if (ok) *reinterpret_cast<uint4*>(y + (size_t)row * K + col) = make_uint4(w[0], w[1], w[2], w[3]);
     } else {
-      quant_store(v, ok, lane, row, col, K, q, s, lds);
+      float o[8];
+      unpack8(make_uint4(w[0], w[1], w[2], w[3]), o);
+      const float sc = e4m3_scale(half_warp_max(amax8(o), lane));
+      if (ok) {
+        *reinterpret_cast<uint2*>(q + (size_t)row * K + col) = quant8(o, sc);
+        if (l == 0) s[(size_t)c * lds + row] = sc;
+      }
     }
   }
 }
@@ -299,19 +331,16 @@ __global__ void __launch_bounds__(kGeluThreads, 1)
     const int st = w - row * steps;
     const int col = lane_col(st, lane);
     const bool ok = col < K;
-    float v[8];
     const uint32_t wd[4] = {cur.x, cur.y, cur.z, cur.w};
+    uint32_t g[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {   // zero inputs (past K) read GELU(0) = 0
-      v[2 * i] = __uint_as_float((uint32_t)lut[wd[i] & 0xFFFFu] << 16);
-      v[2 * i + 1] = __uint_as_float((uint32_t)lut[wd[i] >> 16] << 16);
-    }
+    for (int i = 0; i < 4; ++i)   // zero inputs (past K) read GELU(0) = 0
+      g[i] = (uint32_t)lut[wd[i] & 0xFFFFu] | ((uint32_t)lut[wd[i] >> 16] << 16);
     if (y) {   // bf16 output (may be f itself: each lane reads its 8 values before writing them)
-      if (ok)
-        *reinterpret_cast<uint4*>(y + (size_t)row * ldf + col) =
-            make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]), pack_bf16x2(v[4], v[5]),
-                       pack_bf16x2(v[6], v[7]));
+      if (ok) *reinterpret_cast<uint4*>(y + (size_t)row * ldf + col) = make_uint4(g[0], g[1], g[2], g[3]);
     } else {
+      float v[8];
+      unpack8(make_uint4(g[0], g[1], g[2], g[3]), v);
       quant_store(v, ok, lane, row, col, K, q, s, lds);
     }
     cur = nxt;
@@ -587,28 +616,27 @@ template <int IT>
 static void ln_launch(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* g,
                       const __nv_bfloat16* b, int M, int K, double eps, uint8_t* q, float* s, int lds,
                       __nv_bfloat16* y, cudaStream_t st) {
+  const dim3 grid((unsigned)((M + kLnRows - 1) / kLnRows)), block(16 * kLnRows);
   if (y)
-    launch_pdl(ln_quant_kernel<IT, true>, dim3((unsigned)((M + kLnRows - 1) / kLnRows)), dim3(32 * kLnRows), 0, st,
-               x, ldx, g, b, M, K, eps, q, s, lds, y);
+    launch_pdl(ln_quant_kernel<IT, true>, grid, block, 0, st, x, ldx, g, b, M, K, eps, q, s, lds, y);
   else
-    launch_pdl(ln_quant_kernel<IT, false>, dim3((unsigned)((M + kLnRows - 1) / kLnRows)), dim3(32 * kLnRows), 0, st,
-               x, ldx, g, b, M, K, eps, q, s, lds, y);
+    launch_pdl(ln_quant_kernel<IT, false>, grid, block, 0, st, x, ldx, g, b, M, K, eps, q, s, lds, y);
 }
 
 cudaError_t launch_ln(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,
                       int M, int K, double eps, uint8_t* q, float* s, int lds, __nv_bfloat16* y,
                       cudaStream_t st) {
   if (M == 0) return cudaSuccess;
-  const int it = (K + 255) / 256;
-  switch (it) {
+  const int chunks = (K + 127) / 128;
+  switch (chunks) {
 #define VITQ_LN_CASE(N) \
   case N: ln_launch<N>(x, ldx, gamma, beta, M, K, eps, q, s, lds, y, st); break;
     VITQ_LN_CASE(1) VITQ_LN_CASE(2) VITQ_LN_CASE(3) VITQ_LN_CASE(4) VITQ_LN_CASE(5)
-    VITQ_LN_CASE(6) VITQ_LN_CASE(7) VITQ_LN_CASE(8) VITQ_LN_CASE(9) VITQ_LN_CASE(10)
-    VITQ_LN_CASE(11) VITQ_LN_CASE(12) VITQ_LN_CASE(13) VITQ_LN_CASE(14) VITQ_LN_CASE(15)
-    VITQ_LN_CASE(16) VITQ_LN_CASE(17) VITQ_LN_CASE(18)
+    VITQ_LN_CASE(6) VITQ_LN_CASE(7) VITQ_LN_CASE(8) VITQ_LN_CASE(9)
 #undef VITQ_LN_CASE
-    default: return cudaErrorInvalidValue;
+    default:
+      if (chunks > kLnMaxChunks) return cudaErrorInvalidValue;
+      ln_launch<0>(x, ldx, gamma, beta, M, K, eps, q, s, lds, y, st);
   }
   return cudaGetLastError();
 }

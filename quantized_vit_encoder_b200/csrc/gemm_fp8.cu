@@ -196,23 +196,6 @@ __device__ void gemm_mma(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base, int 
   }
 }
 
-__device__ __forceinline__ uint64_t pack2(float lo, float hi) {
-  uint64_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
-}
-__device__ __forceinline__ float2 unpack2(uint64_t v) {
-  float2 f;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
-  return f;
-}
-// acc (two fp32 lanes) += p * s, one packed FMA.
-__device__ __forceinline__ uint64_t fma2(uint64_t p, uint64_t s, uint64_t acc) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(p), "l"(s), "l"(acc));
-  return d;
-}
-
 template <int BN, bool kPair>
 __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base, const GemmArgs& g,
                               const CUtensorMap* tmC, const CUtensorMap* tmR, int tiles_m, int tiles_n,
@@ -271,7 +254,7 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
         sa_next = row_ok ? __ldg(sa_ptr + (size_t)(kb + 1) * g.ldsA) : 0.f;
         sw_next = col_ok ? __ldg(sw_ptr + kb + 1) : 0.f;
       }
-      const uint64_t s2 = pack2(scale, scale);
+      const uint64_t s2 = f2pack(scale, scale);
       if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(4, cnt);  // epilogue: waiting for partial
       const bool ok = mbar_wait(sm.tfull(buf), aph, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
@@ -286,9 +269,9 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          acc[h * 32 + j] = fma2(pack2(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1])), s2,
+          acc[h * 32 + j] = ffma2(f2pack(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1])), s2,
                                  acc[h * 32 + j]);
-          acc[h * 32 + 16 + j] = fma2(pack2(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1])), s2,
+          acc[h * 32 + 16 + j] = ffma2(f2pack(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1])), s2,
                                       acc[h * 32 + 16 + j]);
         }
       }
@@ -323,7 +306,7 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
         float v[8];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-          const float2 f = unpack2(acc[c8 * 4 + i]);
+          const float2 f = f2unpack(acc[c8 * 4 + i]);
           v[2 * i] = f.x;
           v[2 * i + 1] = f.y;
         }
