@@ -78,6 +78,11 @@ constexpr int kPolyMod = kPolyEvery > 0 ? kPolyEvery : 1;
 #define VITQ_ATTN_TURN_AT 5
 #endif
 constexpr int kTurnAt = VITQ_ATTN_TURN_AT;
+// Whether the two tiles' softmax warps of one SMSP take turns for the exponentials.
+#ifndef VITQ_ATTN_TURNS
+#define VITQ_ATTN_TURNS 1
+#endif
+constexpr bool kTakeTurns = VITQ_ATTN_TURNS != 0;
 
 struct AttnArgs {
   const __nv_bfloat16* qkv;
@@ -339,7 +344,7 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
     // The softmax warps of the two tiles on one SMSP take turns for the
     // exponentials (A(j), B(j), A(j+1), ...): MUFU serves one tile at full rate
     // while the other reads its next scores and waits for its P.V.
-    if (n_q == 2 && (x == 1 || j > 0)) {
+    if (kTakeTurns && n_q == 2 && (x == 1 || j > 0)) {
       ok = mbar_wait(sm.turn(1 - x, quad), (uint32_t)(x == 1 ? j : j - 1) & 1u, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
     }
@@ -372,7 +377,7 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
       *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
       // hand the turn to the other tile a little before the end, so that its
       // exponentials start while these finish (hides the hand-over latency)
-      if (c == kTurnAt && n_q == 2 && !(x == 1 && j == n_kv - 1)) {
+      if (kTakeTurns && c == kTurnAt && n_q == 2 && !(x == 1 && j == n_kv - 1)) {
         __syncwarp();
         if (lane == 0) mbar_arrive(sm.turn(x, quad));
       }

@@ -42,66 +42,76 @@ __device__ __forceinline__ float e4m3_scale(float amax) {
   return __fdiv_rn(amax, kE4M3Max);
 }
 
+// Four fp32 values -> four E4M3 codes in one word (round to nearest even,
+// saturate to +-448), value i in byte i.
+__device__ __forceinline__ uint32_t cvt4_e4m3(float a0, float a1, float a2, float a3) {
+  uint32_t w;
+  asm("{.reg .b16 l, h; cvt.rn.satfinite.e4m3x2.f32 l, %2, %1; cvt.rn.satfinite.e4m3x2.f32 h, %4, %3;"
+      " mov.b32 %0, {l, h};}"
+      : "=r"(w) : "f"(a0), "f"(a1), "f"(a2), "f"(a3));
+  return w;
+}
+
+// E4M3 codes of fl32(v_i / s) by IEEE division (the rare cases of quant8).
+__device__ __noinline__ uint2 quant8_divide(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
+                                            float v7, float s) {
+  return make_uint2(cvt4_e4m3(__fdiv_rn(v0, s), __fdiv_rn(v1, s), __fdiv_rn(v2, s), __fdiv_rn(v3, s)),
+                    cvt4_e4m3(__fdiv_rn(v4, s), __fdiv_rn(v5, s), __fdiv_rn(v6, s), __fdiv_rn(v7, s)));
+}
+
 // E4M3 codes of 8 values of one group, equal to code(fl32(y / s)) without a
 // division.  r = rcp.approx(s) is within 1 ulp of 1/s, so rl = r - 64 ulps
 // <= 1/s <= r + 64 ulps = rh.  For y >= 0, y rl <= y / s <= y rh, and rounding
 // to fp32 and then to E4M3 is monotone, so code(fl(y rl)) <= code(fl(y / s))
 // <= code(fl(y rh)) (mirrored for y < 0): where the outer codes agree, they are
-// the answer.  A pair where they differ (about 2^-12 of pairs) divides exactly.
-// A scale below the fp32 normal range (amax < 448 * 2^-126) has no finite
-// reciprocal; those groups always divide exactly.
+// the answer.  A group where they differ (about 2^-10 of groups) divides
+// exactly.  A scale below the fp32 normal range (amax < 448 * 2^-126), or an
+// infinite or NaN one, divides exactly; a zero scale gives zero codes.
 __device__ __forceinline__ uint2 quant8(const float (&v)[8], float s) {
-  uint32_t w[2] = {0u, 0u};
   if (s >= 1.17549435e-38f && s <= 1e36f) {   // normal, with a normal reciprocal
     float r;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(s));
     const uint32_t rb = __float_as_uint(r);
     const uint64_t rl = f2pack(__uint_as_float(rb - 64u), __uint_as_float(rb - 64u));
     const uint64_t rh = f2pack(__uint_as_float(rb + 64u), __uint_as_float(rb + 64u));
-    uint32_t lo[4], hi[4];
+    float a[8], b[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint64_t x = f2pack(v[2 * i], v[2 * i + 1]);
-      const float2 a = f2unpack(fmul2(x, rl)), b = f2unpack(fmul2(x, rh));
-      lo[i] = cvt_e4m3x2(a.x, a.y);
-      hi[i] = cvt_e4m3x2(b.x, b.y);
+      const float2 p = f2unpack(fmul2(x, rl)), q = f2unpack(fmul2(x, rh));
+      a[2 * i] = p.x;
+      a[2 * i + 1] = p.y;
+      b[2 * i] = q.x;
+      b[2 * i + 1] = q.y;
     }
-    w[0] = __byte_perm(lo[0], lo[1], 0x5410);
-    w[1] = __byte_perm(lo[2], lo[3], 0x5410);
-    const uint32_t h0 = __byte_perm(hi[0], hi[1], 0x5410), h1 = __byte_perm(hi[2], hi[3], 0x5410);
-    if ((w[0] != h0) | (w[1] != h1)) {   // rare: a pair straddles an E4M3 rounding boundary
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (lo[i] != hi[i]) lo[i] = cvt_e4m3x2(__fdiv_rn(v[2 * i], s), __fdiv_rn(v[2 * i + 1], s));
-      }
-      w[0] = __byte_perm(lo[0], lo[1], 0x5410);
-      w[1] = __byte_perm(lo[2], lo[3], 0x5410);
-    }
-  } else if (s > 0.f) {
-    uint32_t c[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) c[i] = cvt_e4m3x2(__fdiv_rn(v[2 * i], s), __fdiv_rn(v[2 * i + 1], s));
-    w[0] = __byte_perm(c[0], c[1], 0x5410);
-    w[1] = __byte_perm(c[2], c[3], 0x5410);
+    uint2 w = make_uint2(cvt4_e4m3(a[0], a[1], a[2], a[3]), cvt4_e4m3(a[4], a[5], a[6], a[7]));
+    const uint32_t h0 = cvt4_e4m3(b[0], b[1], b[2], b[3]), h1 = cvt4_e4m3(b[4], b[5], b[6], b[7]);
+    if ((w.x != h0) | (w.y != h1))   // rare: a value straddles an E4M3 rounding boundary
+      w = quant8_divide(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7], s);
+    return w;
   }
-  return make_uint2(w[0], w[1]);
+  if (s != 0.f) return quant8_divide(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7], s);
+  return make_uint2(0u, 0u);
 }
 
-// Max of |v| over 8 values (NaN ignored, like fmaxf).
-__device__ __forceinline__ float amax8(const float (&v)[8]) {
-  const float a = fmax3(fmax3(fabsf(v[0]), fabsf(v[1]), fabsf(v[2])), fmax3(fabsf(v[3]), fabsf(v[4]), fabsf(v[5])),
-                        fmaxf(fabsf(v[6]), fabsf(v[7])));
-  return a == a ? a : 0.f;
+// Max of |x| over 8 bf16 values (one uint4), as a bf16 bit pattern: the
+// magnitudes of bf16 values order like their bit patterns with the sign
+// cleared, so a packed 16-bit integer max finds it.  A NaN input wins (and
+// makes the group's scale NaN, as the IEEE definition of the max does).
+__device__ __forceinline__ uint32_t amax_bits8(const uint4& u) {
+  uint32_t m;
+  asm("{.reg .b32 t0, t1; max.u16x2 t0, %1, %2; max.u16x2 t1, %3, %4; max.u16x2 %0, t0, t1;}"
+      : "=r"(m)
+      : "r"(u.x & 0x7FFF7FFFu), "r"(u.y & 0x7FFF7FFFu), "r"(u.z & 0x7FFF7FFFu), "r"(u.w & 0x7FFF7FFFu));
+  return max(m & 0xFFFFu, m >> 16);
 }
 
-// Max over each half warp of non-negative values: lanes 0-15 get the max of
-// lanes 0-15, lanes 16-31 that of lanes 16-31 (non-negative floats order like
-// their bit patterns).  All 32 lanes must take part.
-__device__ __forceinline__ float half_warp_max(float a, int lane) {
-  const uint32_t u = __float_as_uint(a);
-  const uint32_t m0 = __reduce_max_sync(0xffffffffu, lane < 16 ? u : 0u);
-  const uint32_t m1 = __reduce_max_sync(0xffffffffu, lane < 16 ? 0u : u);
-  return __uint_as_float(lane < 16 ? m0 : m1);
+// Max over each half warp of bf16 bit patterns, as a float: lanes 0-15 get the
+// max of lanes 0-15, lanes 16-31 that of lanes 16-31.  All 32 lanes must take part.
+__device__ __forceinline__ float half_warp_max_bits(uint32_t m, int lane) {
+  const uint32_t m0 = __reduce_max_sync(0xffffffffu, lane < 16 ? m : 0u);
+  const uint32_t m1 = __reduce_max_sync(0xffffffffu, lane < 16 ? 0u : m);
+  return __uint_as_float((lane < 16 ? m0 : m1) << 16);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float (&v)[8]) {
@@ -122,11 +132,14 @@ __device__ __forceinline__ void load8_bf16(const __nv_bfloat16* p, float (&v)[8]
 __device__ __forceinline__ int lane_col(int step, int lane) { return step * 256 + lane * 8; }
 
 // Group amax over the half warp, scale, codes and scale store for one step
-// (lane layout of lane_col; all 32 lanes take part).
-__device__ __forceinline__ void quant_store(const float (&v)[8], bool ok, int lane, int row, int col, int K,
+// (lane layout of lane_col; all 32 lanes take part).  raw: the lane's 8 bf16
+// values (zeros past K).
+__device__ __forceinline__ void quant_store(const uint4& raw, bool ok, int lane, int row, int col, int K,
                                             uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
-  const float sc = e4m3_scale(half_warp_max(amax8(v), lane));
+  const float sc = e4m3_scale(half_warp_max_bits(amax_bits8(raw), lane));
   if (ok) {
+    float v[8];
+    unpack8(raw, v);
     *reinterpret_cast<uint2*>(q + (size_t)row * K + col) = quant8(v, sc);
     if ((lane & 15) == 0) s[(size_t)(col >> 7) * lds + row] = sc;
   }
@@ -152,21 +165,20 @@ __global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ x, int M, int
 #pragma unroll
   for (int it = 0; it < ITERS; ++it) {
     const int col = lane_col(it, lane);
-    float v[8];
-    unpack8(raw[it], v);
-    quant_store(v, col < K, lane, row, col, K, q, s, lds);
+    quant_store(raw[it], col < K, lane, row, col, K, q, s, lds);
   }
 }
 
 // --------------------------------------------------------- LayerNorm + quant
 // A half warp per row (lane l of the half holds columns 128c + 8l, so each
 // 128-column group is one chunk c across the half warp), eight rows per CTA;
-// gamma and beta are staged once per CTA in shared memory.  The
-// statistics are exact fp64 sums of the bf16 inputs (sum and sum of squares).
-// The normalised value y = (x - mean) rstd gamma + beta is evaluated in fp32;
-// its error is below (|y| + 2|beta|) 2^-20 + 2^-126, and where y minus and
-// plus that bound round to the same bf16 value, that value is the rounding of
-// the exact y.  Elsewhere (about 2^-11 of the pairs) y is recomputed in fp64.
+// gamma, beta and the bracket term below are staged once per CTA in shared
+// memory as fp32.  The statistics are exact fp64 sums of the bf16 inputs (sum
+// and sum of squares).  The normalised value y = (x - mean) rstd gamma + beta
+// is evaluated in fp32; its error is below e = (|y| + 2|beta|) 2^-20 + 2^-126,
+// and where y - e and y + e round to the same bf16 value, that value is the
+// rounding of the exact y.  Elsewhere (about 2^-11 of the pairs) y is
+// recomputed in fp64.
 
 // bf16 pair of ((x - mean) rstd gamma + beta) evaluated in fp64.
 __device__ __noinline__ uint32_t ln_pair_fp64(float x0, float x1, float g0, float g1, float b0, float b1,
@@ -186,14 +198,35 @@ __global__ void __launch_bounds__(16 * kLnRows, 6)
     ln_quant_kernel(const __nv_bfloat16* __restrict__ x, int ldx, const __nv_bfloat16* __restrict__ gamma,
                     const __nv_bfloat16* __restrict__ beta, int M, int K, double eps,
                     uint8_t* __restrict__ q, float* __restrict__ s, int lds, __nv_bfloat16* __restrict__ y) {
-  constexpr int kSm = ITERS > 0 ? ITERS : kLnMaxChunks;
-  __shared__ uint4 sg[kSm * 16], sb[kSm * 16];
+  // per column: gamma, beta, (2|beta| 2^-20 + 2^-126), as fp32 (dynamic shared memory,
+  // nch * 1536 bytes).  Columns 128c + 8l + 4h .. +3 sit in float4 (2c + h) * 16 + l, so
+  // the 16 lanes of a half warp read 16 consecutive float4.
+  extern __shared__ float4 ln_smem[];
   const int nch = ITERS > 0 ? ITERS : (K + 127) >> 7;
+  float4* sg = ln_smem;
+  float4* sb = ln_smem + nch * 32;
+  float4* se = ln_smem + 2 * nch * 32;
   pdl_trigger();
   for (int i = threadIdx.x; i < nch * 16; i += blockDim.x) {
     const int col = i * 8;
-    sg[i] = col < K ? *reinterpret_cast<const uint4*>(gamma + col) : make_uint4(0, 0, 0, 0);
-    sb[i] = col < K ? *reinterpret_cast<const uint4*>(beta + col) : make_uint4(0, 0, 0, 0);
+    float g[8], b[8];
+    if (col < K) {
+      load8_bf16(gamma + col, g);
+      load8_bf16(beta + col, b);
+    } else {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) g[k] = b[k] = 0.f;
+    }
+    const int j0 = ((i >> 4) * 2) * 16 + (i & 15), j1 = j0 + 16;
+    sg[j0] = make_float4(g[0], g[1], g[2], g[3]);
+    sg[j1] = make_float4(g[4], g[5], g[6], g[7]);
+    sb[j0] = make_float4(b[0], b[1], b[2], b[3]);
+    sb[j1] = make_float4(b[4], b[5], b[6], b[7]);
+    float e[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) e[k] = fmaf(fabsf(b[k]), 0x1p-19f, 0x1p-126f);
+    se[j0] = make_float4(e[0], e[1], e[2], e[3]);
+    se[j1] = make_float4(e[4], e[5], e[6], e[7]);
   }
   __syncthreads();
   pdl_wait();   // x may be the previous kernel's output
@@ -236,20 +269,23 @@ __global__ void __launch_bounds__(16 * kLnRows, 6)
   for (int c = 0; c < nch; ++c) {
     const int col = c * 128 + l * 8;
     const bool ok = row_ok && col < K;
-    float v[8], g[8], b[8];
+    float v[8];
     unpack8(load_chunk(c), v);
-    unpack8(sg[c * 16 + l], g);
-    unpack8(sb[c * 16 + l], b);
-    uint32_t w[4];
+    const int j0 = c * 32 + l, j1 = j0 + 16;
+    const float4 g0 = sg[j0], g1 = sg[j1], b0 = sb[j0], b1 = sb[j1], e0 = se[j0], e1 = se[j1];
+    const float g[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+    const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+    const float eb[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+    uint4 wq;
+    uint32_t* w = reinterpret_cast<uint32_t*>(&wq);
     uint32_t slow = 0u;   // pairs whose bracket straddles a bf16 rounding boundary
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const uint64_t t = fmul2(fadd2(fadd2(f2pack(v[2 * i], v[2 * i + 1]), nmh), nml), rr);
       const uint64_t yy = ffma2(t, f2pack(g[2 * i], g[2 * i + 1]), f2pack(b[2 * i], b[2 * i + 1]));
       const float2 yf = f2unpack(yy);
-      const float e0 = fmaf(fabsf(yf.x), 0x1p-20f, fmaf(fabsf(b[2 * i]), 0x1p-19f, 0x1p-126f));
-      const float e1 = fmaf(fabsf(yf.y), 0x1p-20f, fmaf(fabsf(b[2 * i + 1]), 0x1p-19f, 0x1p-126f));
-      const uint64_t e = f2pack(e0, e1);
+      const uint64_t e = ffma2(f2pack(fabsf(yf.x), fabsf(yf.y)), f2pack(0x1p-20f, 0x1p-20f),
+                               f2pack(eb[2 * i], eb[2 * i + 1]));
       const uint32_t lo = bf16x2_of(ffma2(e, f2pack(-1.f, -1.f), yy)), hi = bf16x2_of(fadd2(yy, e));
       slow |= (uint32_t)(lo != hi) << i;
       w[i] = lo;
@@ -261,12 +297,12 @@ __global__ void __launch_bounds__(16 * kLnRows, 6)
           w[i] = ln_pair_fp64(v[2 * i], v[2 * i + 1], g[2 * i], g[2 * i + 1], b[2 * i], b[2 * i + 1], mean, rstd);
     }
     if (kOutBf16) {   // bf16 output (the bf16 blocks and mergers)
-      if (ok) *reinterpret_cast<uint4*>(y + (size_t)row * K + col) = make_uint4(w[0], w[1], w[2], w[3]);
+      if (ok) *reinterpret_cast<uint4*>(y + (size_t)row * K + col) = wq;
     } else {
-      float o[8];
-      unpack8(make_uint4(w[0], w[1], w[2], w[3]), o);
-      const float sc = e4m3_scale(half_warp_max(amax8(o), lane));
+      const float sc = e4m3_scale(half_warp_max_bits(amax_bits8(wq), lane));
       if (ok) {
+        float o[8];
+        unpack8(wq, o);
         *reinterpret_cast<uint2*>(q + (size_t)row * K + col) = quant8(o, sc);
         if (l == 0) s[(size_t)c * lds + row] = sc;
       }
@@ -298,7 +334,10 @@ constexpr int kGeluThreads = 1024;
 constexpr size_t kGeluSmem = 65536 * 2;
 
 // Persistent: one CTA per SM copies the table into shared memory, then each warp
-// takes (row, 256-column step) items in turn (lane layout of lane_col).
+// takes (row, 256-column step) items w, w + W, w + 2W, ... (W = warps in the
+// grid; lane layout of lane_col), stepping (row, step) incrementally.  The next
+// item's 8 inputs per lane are loaded before the current item is processed, so
+// the load latency overlaps the work.
 __global__ void __launch_bounds__(kGeluThreads, 1)
     gelu_quant_kernel(const __nv_bfloat16* f, int M, int K, int ldf, uint8_t* __restrict__ q,
                       float* __restrict__ s, int lds, __nv_bfloat16* y) {
@@ -313,37 +352,39 @@ __global__ void __launch_bounds__(kGeluThreads, 1)
   __syncthreads();
   pdl_wait();
   const int steps = (K + 255) / 256;
-  const int items = M * steps;
   const int lane = threadIdx.x & 31;
   const int warps = gridDim.x * (kGeluThreads / 32);
-  // each warp walks items w, w + warps, ...; the next item's 8 inputs per lane are
-  // loaded before the current item is processed, so the load latency overlaps the work
-  auto load = [&](int w) {
-    const int row = w / steps, col = lane_col(w - row * steps, lane);
-    return (w < items && col < K) ? *reinterpret_cast<const uint4*>(f + (size_t)row * ldf + col)
-                                  : make_uint4(0u, 0u, 0u, 0u);
+  const int w0 = blockIdx.x * (kGeluThreads / 32) + (threadIdx.x >> 5);
+  const int drow = warps / steps, dst_ = warps - drow * steps;   // item stride as (rows, steps)
+  int row = w0 / steps, st = w0 - row * steps;
+  auto load = [&](int r, int t) {
+    const int col = lane_col(t, lane);
+    return (r < M && col < K) ? *reinterpret_cast<const uint4*>(f + (size_t)r * ldf + col) : make_uint4(0u, 0u, 0u, 0u);
   };
-  int w = blockIdx.x * (kGeluThreads / 32) + (threadIdx.x >> 5);
-  uint4 cur = load(w);
-  for (; w < items; w += warps) {
-    const uint4 nxt = load(w + warps);
-    const int row = w / steps;
-    const int st = w - row * steps;
+  uint4 cur = load(row, st);
+  while (row < M) {
+    int nrow = row + drow, nst = st + dst_;
+    if (nst >= steps) {
+      nst -= steps;
+      ++nrow;
+    }
+    const uint4 nxt = load(nrow, nst);
     const int col = lane_col(st, lane);
     const bool ok = col < K;
     const uint32_t wd[4] = {cur.x, cur.y, cur.z, cur.w};
-    uint32_t g[4];
+    uint4 g;
+    uint32_t* gv = reinterpret_cast<uint32_t*>(&g);
 #pragma unroll
     for (int i = 0; i < 4; ++i)   // zero inputs (past K) read GELU(0) = 0
-      g[i] = (uint32_t)lut[wd[i] & 0xFFFFu] | ((uint32_t)lut[wd[i] >> 16] << 16);
+      gv[i] = (uint32_t)lut[wd[i] & 0xFFFFu] | ((uint32_t)lut[wd[i] >> 16] << 16);
     if (y) {   // bf16 output (may be f itself: each lane reads its 8 values before writing them)
-      if (ok) *reinterpret_cast<uint4*>(y + (size_t)row * ldf + col) = make_uint4(g[0], g[1], g[2], g[3]);
+      if (ok) *reinterpret_cast<uint4*>(y + (size_t)row * ldf + col) = g;
     } else {
-      float v[8];
-      unpack8(make_uint4(g[0], g[1], g[2], g[3]), v);
-      quant_store(v, ok, lane, row, col, K, q, s, lds);
+      quant_store(g, ok, lane, row, col, K, q, s, lds);
     }
     cur = nxt;
+    row = nrow;
+    st = nst;
   }
 }
 
@@ -617,10 +658,10 @@ static void ln_launch(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* g,
                       const __nv_bfloat16* b, int M, int K, double eps, uint8_t* q, float* s, int lds,
                       __nv_bfloat16* y, cudaStream_t st) {
   const dim3 grid((unsigned)((M + kLnRows - 1) / kLnRows)), block(16 * kLnRows);
-  if (y)
-    launch_pdl(ln_quant_kernel<IT, true>, grid, block, 0, st, x, ldx, g, b, M, K, eps, q, s, lds, y);
-  else
-    launch_pdl(ln_quant_kernel<IT, false>, grid, block, 0, st, x, ldx, g, b, M, K, eps, q, s, lds, y);
+  const size_t smem = (size_t)((K + 127) / 128) * 1536;
+  auto kern = y ? ln_quant_kernel<IT, true> : ln_quant_kernel<IT, false>;
+  if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  launch_pdl(kern, grid, block, smem, st, x, ldx, g, b, M, K, eps, q, s, lds, y);
 }
 
 cudaError_t launch_ln(const __nv_bfloat16* x, int ldx, const __nv_bfloat16* gamma, const __nv_bfloat16* beta,

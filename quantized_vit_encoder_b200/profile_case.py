@@ -3,9 +3,12 @@
     python -m quantized_vit_encoder_b200.profile_case STAGE [--iters N]
 
 STAGE: attention | gemm_qkv | gemm_proj | gemm_fc1 | gemm_fc2 | bf16_qkv | bf16_proj | bf16_fc1 |
-       bf16_fc2 | ln_quant | ln_quant_merger | quant_act | gelu_quant | rope | block.
-Device memory stays below 0.5 GB; each iteration is one launch of the stage's
-kernel (block: the ten launches of one block).
+       bf16_fc2 | ln_quant | ln_quant_merger | quant_act | gelu_quant | rope | block | tower.
+Device memory stays below 0.5 GB except for tower (the 27 blocks' and 4 mergers'
+weights, about 1 GB); each iteration is one launch of the stage's kernel (block:
+the ten launches of one block; tower: the 288 launches of one tower pass).  The
+last iteration runs inside the NVTX range "last_iter", so a profiler can select
+exactly its launches (ncu --nvtx --nvtx-include "last_iter/").
 """
 from __future__ import annotations
 
@@ -32,7 +35,14 @@ def main():
     pos, cu = vitq.positions(list(W.grids), dev)
     cs = vitq.rope_table(pos)
     t = blk.t
-    if a.stage == "block":
+    if a.stage == "tower":
+        blocks = [vitq.DeviceBlock(wl.block_params(wl.block_seed(W, b)), dev) for b in range(wl.N_BLOCKS)]
+        mergers = [vitq.DeviceMerger(wl.merger_params(wl.merger_seed(W, m)), dev) for m in range(4)]
+        tower = vitq.DeviceTower(blocks, mergers)
+        ws = vitq.workspace(vitq.tower_workspace_bytes(n, 1), dev)
+        xt = x.clone()
+        run = lambda: vitq.tower_forward_(tower, xt.copy_(x), list(W.grids), ws)  # noqa: E731
+    elif a.stage == "block":
         ws = vitq.workspace(vitq.block_workspace_bytes(n), dev)
         run = lambda: vitq.block_forward_(blk, x, cu, n, cs, ws)  # noqa: E731
     elif a.stage == "attention":
@@ -72,8 +82,12 @@ def main():
         run = lambda: vitq.rope2d_(qkv, cs)  # noqa: E731
     else:
         raise SystemExit(f"unknown stage {a.stage}")
-    for _ in range(a.iters):
+    for _ in range(a.iters - 1):
         run()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("last_iter")
+    run()
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     assert vitq.device_error() == 0
     print(f"{a.stage}: {a.iters} iterations ok")
