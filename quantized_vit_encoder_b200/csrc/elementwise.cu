@@ -149,7 +149,7 @@ __device__ __forceinline__ void quant_store(const uint4& raw, bool ok, int lane,
 // One warp per row; every load of the row is issued before any use.
 
 template <int ITERS>
-__global__ void quant_act_kernel(const __nv_bfloat16* __restrict__ x, int M, int K, int ldx,
+__global__ void __launch_bounds__(128, 12) quant_act_kernel(const __nv_bfloat16* __restrict__ x, int M, int K, int ldx,
                                  uint8_t* __restrict__ q, float* __restrict__ s, int lds) {
   pdl_trigger();
   pdl_wait();
@@ -453,69 +453,50 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int n, double
   cs[(size_t)t * 72 + 36 + j] = (float)sn;
 }
 
-// One CTA per token, one thread per 8-element chunk.  Chunks 0..287 are the
-// token's q and k heads (9 per head): x'_j = x_j c_j - x_(j+36) s_j,
-// x'_(j+36) = x_(j+36) c_j + x_j s_j; the partner elements of chunk cc live in
-// two neighbouring chunks A (elements 4..7) and B (elements 0..3).  Chunks
-// 288..431 are the v heads, converted to fp16 in place when v_to_f16 (round to
-// nearest: exact for 2^-14 <= |v| < 65504, within 2^-25 below).  All reads happen before the barrier and all
-// writes after it, so the in-place update never reads a rotated value.
-__global__ void __launch_bounds__(432) rope_apply_kernel(__nv_bfloat16* __restrict__ qkv,
-                                                         const float* __restrict__ cs, int v_to_f16) {
+// One thread per work item, 432 items per token, no barrier: items 0..287 are
+// (q/k head slot, group of four rotary pairs): the thread reads x_j .. x_(j+3)
+// and their partners x_(j+36) .. x_(j+39) (8 bytes each) and writes both,
+// x'_j = x_j c_j - x_(j+36) s_j and x'_(j+36) = x_(j+36) c_j + x_j s_j, so no
+// thread reads what another writes.  Items 288..431 are the 8-element chunks of
+// the v heads, converted to fp16 in place when v_to_f16 (round to nearest:
+// exact for 2^-14 <= |v| < 65504, within 2^-25 below).
+constexpr int kRopeItems = 432;
+
+__global__ void __launch_bounds__(256) rope_apply_kernel(__nv_bfloat16* __restrict__ qkv,
+                                                         const float* __restrict__ cs, int n, int v_to_f16) {
   pdl_trigger();
   pdl_wait();
-  const int t = blockIdx.x;
-  const int c = threadIdx.x;
+  const long long g = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const int t = (int)(g / kRopeItems), w = (int)(g - (long long)t * kRopeItems);
+  if (t >= n) return;
   __nv_bfloat16* base = qkv + (size_t)t * 3456;
-  uint4 out = make_uint4(0, 0, 0, 0);
-  __nv_bfloat16* dst = nullptr;
-  if (c < 288) {
-    const int slot = c / 9, cc = c - slot * 9;
-    const __nv_bfloat16* head = base + slot * 72;
-    int ca, cb, k0, k1;   // partner chunks, cos/sin offsets of elements 0..3 and 4..7
-    if (cc < 4) {
-      ca = cc + 4; cb = cc + 5; k0 = 8 * cc; k1 = 8 * cc + 4;
-    } else if (cc == 4) {
-      ca = 8; cb = 0; k0 = 32; k1 = 0;
-    } else {
-      ca = cc - 5; cb = cc - 4; k0 = 8 * cc - 36; k1 = 8 * cc - 32;
-    }
-    float x[8], pa[8], pb[8];
-    load8_bf16(head + cc * 8, x);
-    load8_bf16(head + ca * 8, pa);
-    load8_bf16(head + cb * 8, pb);
-    const float* tc = cs + (size_t)t * 72;
-    const float4 c0 = __ldg(reinterpret_cast<const float4*>(tc + k0));
-    const float4 c1 = __ldg(reinterpret_cast<const float4*>(tc + k1));
-    const float4 s0 = __ldg(reinterpret_cast<const float4*>(tc + 36 + k0));
-    const float4 s1 = __ldg(reinterpret_cast<const float4*>(tc + 36 + k1));
-    const float cv[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-    const float pv[8] = {pa[4], pa[5], pa[6], pa[7], pb[0], pb[1], pb[2], pb[3]};
-    float o[8];
+  if (w < 288) {
+    const int slot = w / 9, p = w - slot * 9, j = 4 * p;
+    uint2* lo = reinterpret_cast<uint2*>(base + slot * 72 + j);
+    uint2* hi = reinterpret_cast<uint2*>(base + slot * 72 + 36 + j);
+    const uint2 a = *lo, b = *hi;
+    const float4 c = __ldg(reinterpret_cast<const float4*>(cs + (size_t)t * 72 + j));
+    const float4 sn = __ldg(reinterpret_cast<const float4*>(cs + (size_t)t * 72 + 36 + j));
+    const float2 a0 = unpack_bf16x2(a.x), a1 = unpack_bf16x2(a.y), b0 = unpack_bf16x2(b.x), b1 = unpack_bf16x2(b.y);
+    const float x[4] = {a0.x, a0.y, a1.x, a1.y}, y[4] = {b0.x, b0.y, b1.x, b1.y};
+    const float cv[4] = {c.x, c.y, c.z, c.w}, sv[4] = {sn.x, sn.y, sn.z, sn.w};
+    float xo[4], yo[4];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const bool first_half = cc < 4 || (cc == 4 && i < 4);   // element j < 36
-      o[i] = first_half ? fmaf(x[i], cv[i], -pv[i] * sv[i]) : fmaf(x[i], cv[i], pv[i] * sv[i]);
+    for (int i = 0; i < 4; ++i) {
+      xo[i] = fmaf(x[i], cv[i], -y[i] * sv[i]);
+      yo[i] = fmaf(y[i], cv[i], x[i] * sv[i]);
     }
-    out.x = pack_bf16x2(o[0], o[1]);
-    out.y = pack_bf16x2(o[2], o[3]);
-    out.z = pack_bf16x2(o[4], o[5]);
-    out.w = pack_bf16x2(o[6], o[7]);
-    dst = base + slot * 72 + cc * 8;
+    *lo = make_uint2(pack_bf16x2(xo[0], xo[1]), pack_bf16x2(xo[2], xo[3]));
+    *hi = make_uint2(pack_bf16x2(yo[0], yo[1]), pack_bf16x2(yo[2], yo[3]));
   } else if (v_to_f16) {
-    dst = base + 2304 + (c - 288) * 8;
+    __nv_bfloat16* dst = base + 2304 + (w - 288) * 8;
     float v[8];
     load8_bf16(dst, v);
     __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
     __half2 h2 = __floats2half2_rn(v[4], v[5]), h3 = __floats2half2_rn(v[6], v[7]);
-    out.x = *reinterpret_cast<uint32_t*>(&h0);
-    out.y = *reinterpret_cast<uint32_t*>(&h1);
-    out.z = *reinterpret_cast<uint32_t*>(&h2);
-    out.w = *reinterpret_cast<uint32_t*>(&h3);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),
+                                                *reinterpret_cast<uint32_t*>(&h2), *reinterpret_cast<uint32_t*>(&h3));
   }
-  __syncthreads();
-  if (dst) *reinterpret_cast<uint4*>(dst) = out;
 }
 
 // --------------------------------------------------------------- positions
@@ -718,7 +699,8 @@ cudaError_t launch_rope_table(const int32_t* pos, int n, double theta, float* cs
 
 cudaError_t launch_rope_apply(__nv_bfloat16* qkv, int n, const float* cs, int v_to_f16, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
-  launch_pdl(rope_apply_kernel, dim3(n), dim3(432), 0, st, qkv, cs, v_to_f16);
+  const long long items = (long long)n * kRopeItems;
+  launch_pdl(rope_apply_kernel, dim3((unsigned)((items + 255) / 256)), dim3(256), 0, st, qkv, cs, n, v_to_f16);
   return cudaGetLastError();
 }
 
