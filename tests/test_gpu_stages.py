@@ -334,3 +334,43 @@ def test_attention_full_6256_sampled_rows(lib):
         p = np.exp(s)
         ref[:, h] = (p / p.sum(1, keepdims=True)) @ t[:, 2, h]
     assert_close(got[rows], onum.bf16_round(ref.reshape(256, -1)), what="attention 6256 sampled")
+
+
+def test_zero_rows_are_no_ops(lib):
+    """Zero rows through every stage entry point: status ok, outputs untouched, no device error."""
+    from quantized_vit_encoder_b200 import vitq
+    L = vitq.load()
+    s = vitq._stream(None)
+    p = vitq._p
+    x = torch.full((4, 1152), 1.5, dtype=torch.bfloat16, device="cuda")
+    f = torch.full((4, 4304), 1.5, dtype=torch.bfloat16, device="cuda")
+    q = torch.full((4, 4304), 7, dtype=torch.uint8, device="cuda")
+    sc = torch.full((34, 4), -1.0, dtype=torch.float32, device="cuda")
+    g = torch.ones(1152, dtype=torch.bfloat16, device="cuda")
+    b = torch.zeros(1152, dtype=torch.bfloat16, device="cuda")
+    w = torch.full((1152, 1152), 3, dtype=torch.uint8, device="cuda")
+    sw = torch.ones((9, 9), dtype=torch.float32, device="cuda")
+    out = torch.full((4, 1152), 2.0, dtype=torch.bfloat16, device="cuda")
+    assert L.vit_quant_act(p(x), 0, 1152, 1152, p(q), p(sc), 4, s) == 0
+    assert L.vit_ln_quant(p(x), 0, 1152, 1152, p(g), p(b), 1e-6, p(q), p(sc), 4, s) == 0
+    assert L.vit_gelu_quant(p(f), 0, 4304, 4304, p(q), p(sc), 4, s) == 0
+    assert L.fp8_block_gemm(p(q), p(sc), 4, p(w), p(sw), None, None, p(out), 0, 1152, 1152, s) == 0
+    cu0 = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert L.vit_attention_varlen(p(f), 0, p(cu0), 0, 0, 0.1, 0, p(out), s) == 0
+    torch.cuda.synchronize()
+    assert vitq.device_error() == 0
+    assert torch.all(q == 7) and torch.all(sc == -1.0) and torch.all(out == 2.0)
+
+
+def test_attention_empty_segment_in_a_packed_batch(lib):
+    """A zero-length segment between two others: its CTAs do nothing, the others are unaffected."""
+    from quantized_vit_encoder_b200 import vitq
+    lens = [5, 0, 7]
+    n = sum(lens)
+    cu = wl.random_cu_seqlens(lens)
+    qkv = bf16((n, 3456), 77, 1.0)
+    ref = ov.attention_varlen(f64(qkv), cu)
+    got = vitq.attention_varlen(qkv.cuda(), torch.tensor(cu, dtype=torch.int32, device="cuda"), max(lens))
+    torch.cuda.synchronize()
+    assert vitq.device_error() == 0
+    assert_close(f64(got), ref, what="attention with an empty segment")
