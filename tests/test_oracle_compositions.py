@@ -1,0 +1,93 @@
+"""Pins of the oracle's compositions (block, tower) against closed forms and invariants.
+
+The stage functions are pinned one by one elsewhere; these tests tie the way the
+oracle wires them together to facts that hold for the method itself:
+
+* a block whose four linear weights are zero reduces to its two residual adds,
+  x2 = bf16(bf16(x + b_proj) + b_fc2) (attention then averages identical v rows,
+  which must give the v bias back exactly);
+* with such blocks the tower state after block b follows that recursion, so the
+  mergers must see the states after blocks 8, 16, 24 and 27 (1-indexed);
+* a block over packed images equals the block over each image alone, bit for bit
+  (every stage is row-wise except attention, which is per segment).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import numerics as nm
+from oracle import vit as ov
+from quantized_vit_encoder_b200 import workloads as wl
+
+pytestmark = pytest.mark.filterwarnings("ignore::RuntimeWarning")
+
+
+def _f64(t):
+    return t.float().double().numpy() if isinstance(t, torch.Tensor) else np.asarray(t, np.float64)
+
+
+def _zero_linear_block(seed):
+    """Block weights with zero linears and the seeded LayerNorm vectors and biases."""
+    p = {k: _f64(v) for k, v in wl.block_params(seed).items()}
+    for name in ("qkv", "proj", "fc1", "fc2"):
+        p[name + "_w"] = np.zeros_like(p[name + "_w"])
+    return ov.quantize_block_weights(p)
+
+
+def test_zero_weight_quantisation_is_all_zero():
+    q, s = ov.quant_weight(np.zeros((256, 384)))
+    assert not q.any() and not s.any()
+
+
+@pytest.mark.parametrize("grids", [[(4, 4)], [(3, 5)], [(2, 2), (4, 6)]])
+def test_block_with_zero_linears_is_its_residual_adds(grids):
+    w = _zero_linear_block(11)
+    pos, cu = ov.packed_positions(grids)
+    n = pos.shape[0]
+    x = _f64(wl.random_bf16((n, 1152), 12, 1.0))
+    x2, st = ov.block_forward(x, w, cu, pos, keep=True)
+    # the qkv projection is its bias on every row, so attention returns the v bias
+    v_b = w["qkv_b"][2304:]
+    assert np.array_equal(st["attn"], np.broadcast_to(v_b, (n, 1152)))
+    x1 = nm.bf16_round(x + w["proj_b"])
+    assert np.array_equal(st["x1"], x1)
+    assert np.array_equal(x2, nm.bf16_round(x1 + w["fc2_b"]))
+
+
+def test_tower_taps_follow_blocks_8_16_24_27(monkeypatch):
+    blocks = [_zero_linear_block(100 + b) for b in range(wl.N_BLOCKS)]
+    mergers = [ov.quantize_merger_weights({k: _f64(v) for k, v in wl.merger_params(200 + t).items()})
+               for t in range(4)]
+    grids = [(2, 2)]
+    x = _f64(wl.random_bf16((4, 1152), 13, 1.0))
+    states = [x]
+    for w in blocks:
+        x1 = nm.bf16_round(states[-1] + w["proj_b"])
+        states.append(nm.bf16_round(x1 + w["fc2_b"]))
+    seen = []
+    real = ov.merger_forward
+
+    def spy(h, m, eps=1e-6, keep=False):
+        seen.append(np.array(h))
+        return real(h, m, eps, keep)
+
+    monkeypatch.setattr(ov, "merger_forward", spy)
+    taps = ov.tower_forward(x, blocks, mergers, grids)
+    assert len(taps) == 4 and len(seen) == 4
+    for h, b in zip(seen, (8, 16, 24, 27)):
+        assert np.array_equal(h, states[b]), f"merger input is not the state after block {b}"
+    for tap, h, m in zip(taps, seen, mergers):
+        assert np.array_equal(tap, real(h, m))
+
+
+def test_block_over_packed_images_equals_each_image_alone():
+    w = ov.quantize_block_weights({k: _f64(v) for k, v in wl.block_params(21).items()})
+    grids = [(4, 2), (3, 3), (2, 6)]
+    pos, cu = ov.packed_positions(grids)
+    x = _f64(wl.random_bf16((pos.shape[0], 1152), 22, 1.0))
+    packed = ov.block_forward(x, w, cu, pos)
+    for i, g in enumerate(grids):
+        a, b = int(cu[i]), int(cu[i + 1])
+        p1, c1 = ov.packed_positions([g])
+        alone = ov.block_forward(x[a:b], w, c1, p1)
+        assert np.array_equal(packed[a:b], alone)
