@@ -108,9 +108,10 @@ int pick_block_n(int M, int N, int num_sms) {
     const int v = std::atoi(env);
     if (v == 128 || v == 256) return v;
   }
-  // 128 x 256 tiles read 25 % fewer operand bytes per output than 128 x 128 (the
-  // GEMMs are bound by operand traffic from L2); narrow outputs keep 128 for
-  // enough tiles per SM.
+  // Every 128-wide K block of a tile costs a fixed ~450-500 cycles beyond its MMA
+  // work (measured), so 128 x 256 tiles, with half as many K blocks per output,
+  // win where N is wide; narrow outputs keep 128 for enough tiles per SM (and
+  // four TMEM partial buffers, which hide the epilogue).
   (void)M;
   (void)num_sms;
   return N > 1536 ? 256 : 128;

@@ -30,9 +30,9 @@ __device__ __forceinline__ uint32_t bf16x2_of(uint64_t v) {
 // ------------------------------------------------ exact block-128 quantisation
 // Group scale fl32(amax / 448) without a division: q0 = fl(amax * R) with
 // R = fl(1/448), then one FMA correction.  For every bf16 amax from 2^-100 to
-// the largest finite bf16 this equals the IEEE quotient (checked exhaustively);
-// every amax here is a bf16 value (the quantised inputs are bf16).  Other
-// values take the IEEE division.
+// the largest finite bf16 this equals the IEEE quotient (each of them checked
+// on the host in exact rational arithmetic); every amax here is a bf16 value
+// (the quantised inputs are bf16).  Other values take the IEEE division.
 __device__ __forceinline__ float e4m3_scale(float amax) {
   if (amax >= 7.88860905e-31f && amax <= 3.38953139e38f) {
     constexpr float R = 1.0f / 448.0f;

@@ -12,7 +12,8 @@
 //     128 rows of A and half of the BN rows of W, and the leader issues
 //     cta_group::2 MMAs that read both CTAs' shared memory and write both
 //     CTAs' TMEM, so each SM fetches 16 + BN/2 x 128 bytes per K block instead
-//     of 16 + BN x 128 (the K loop is bound by that operand supply);
+//     of 16 + BN x 128 (measured slower than single CTAs on the block's
+//     shapes, so it is off unless VITQ_GEMM_PAIR=1);
 //   * warp 0: TMA producer (A and W tiles of 128 K-columns into a multi-stage
 //     128B-swizzled shared-memory ring, zero fill past K / M / N);
 //   * warp 1: MMA issuer, 4 x tcgen05.mma kind::f8f6f4 (K = 32 each) per K
