@@ -398,6 +398,48 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     video_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
     del vws, vx, vx0, vtaps
 
+    # the packed four-image batch (54x18 + 46x136 + 24x38 + 32x32 = 9164 patches, per-image
+    # input scales 0.1 / 1 / 10 / 1) through the same tower, and one block at 16x16 and at
+    # 36x27 (row-major odd grid): the other shapes of the workload set, timed the same way
+    PW = wl.WORKLOADS["tower_packed4"]
+    px0 = wl.make_input(PW).to(dev)
+    px = torch.empty_like(px0)
+    pws4 = vitq.workspace(vitq.tower_workspace_bytes(PW.n_tokens, len(PW.grids)), dev)
+    ptaps = [torch.empty((PW.n_tokens // 4, wl.OUT_HIDDEN), dtype=torch.bfloat16, device=dev) for _ in range(4)]
+
+    def packed_step():
+        px.copy_(px0)
+        vitq.tower_forward_(tower, px, list(PW.grids), pws4, ptaps)
+
+    for _ in range(2):
+        packed_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        packed_step()
+    ev1.record(stream)
+    barrier()
+    packed_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    del pws4, px, px0, ptaps
+    small_blocks = {}
+    for name in ("block_16x16", "block_36x27"):
+        SW = wl.WORKLOADS[name]
+        spos, scu = vitq.positions(list(SW.grids), dev)
+        scs = vitq.rope_table(spos)
+        sx = wl.make_input(SW).to(dev)
+        sws = vitq.workspace(vitq.block_workspace_bytes(SW.n_tokens), dev)
+        smax = max(h * w for h, w in SW.grids)
+        for _ in range(args.warmup):
+            vitq.block_forward_(blk, sx, scu, smax, scs, sws)
+        barrier()
+        ev0.record(stream)
+        for _ in range(nb):
+            vitq.block_forward_(blk, sx, scu, smax, scs, sws)
+        ev1.record(stream)
+        barrier()
+        small_blocks[name] = max_over_ranks(ev0.elapsed_time(ev1) / nb)
+        del sws, sx
+
     # per-kernel device times from a profiled pass of the same step (not the timed one)
     vitq.profile_start()
     for _ in range(2):
@@ -452,6 +494,10 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "mixed_tower_ms": mixed_ms,
         "patch_embed_ms": patch_ms,
         "video_8x32x32_tower_ms": video_ms,
+        "packed4_9164_tower_ms": packed_ms,
+        "packed4_9164_tower_tflops": tower_flops(wl.WORKLOADS["tower_packed4"].grids)["tower"] / packed_ms / 1e9,
+        "block_16x16_ms": small_blocks["block_16x16"],
+        "block_36x27_ms": small_blocks["block_36x27"],
         "roofline": roofline(table, peaks),
         "kernels": {k: {"launches": v["launches"] // 2, "ms_per_step": v["ms"] / 2,
                         "share": v["ms"] / sum(t["ms"] for t in table.values())} for k, v in table.items()},
