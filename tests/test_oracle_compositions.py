@@ -91,3 +91,31 @@ def test_block_over_packed_images_equals_each_image_alone():
         p1, c1 = ov.packed_positions([g])
         alone = ov.block_forward(x[a:b], w, c1, p1)
         assert np.array_equal(packed[a:b], alone)
+
+
+def test_bf16_block_with_zero_linears_is_its_residual_adds():
+    """The bf16 block of the mixed tower has the same residual wiring as the FP8 block."""
+    p = {k: _f64(v) for k, v in wl.block_params(41).items()}
+    for name in ("qkv", "proj", "fc1", "fc2"):
+        p[name + "_w"] = np.zeros_like(p[name + "_w"])
+    pos, cu = ov.packed_positions([(4, 4), (2, 6)])
+    n = pos.shape[0]
+    x = _f64(wl.random_bf16((n, 1152), 42, 1.0))
+    x2 = ov.block_forward_bf16(x, p, cu, pos)
+    x1 = nm.bf16_round(x + p["proj_b"])
+    assert np.array_equal(x2, nm.bf16_round(x1 + p["fc2_b"]))
+
+
+def test_mixed_tower_runs_bf16_then_fp8_blocks(monkeypatch):
+    """tower_forward dispatches each block on its weights: bf16 weights (no FP8 codes) run
+    the bf16 block, quantised weights the FP8 block, in the given order."""
+    calls = []
+    monkeypatch.setattr(ov, "block_forward", lambda h, w, cu, pos, eps=1e-6: calls.append("fp8") or h)
+    monkeypatch.setattr(ov, "block_forward_bf16", lambda h, w, cu, pos, eps=1e-6: calls.append("bf16") or h)
+    monkeypatch.setattr(ov, "merger_forward", lambda h, m, eps=1e-6, keep=False: h[: h.shape[0] // 4])
+    monkeypatch.setattr(ov, "merger_forward_bf16", lambda h, m, eps=1e-6, keep=False: h[: h.shape[0] // 4])
+    bf16_w, fp8_w = {"qkv_w": None}, {"qkv_q": None}
+    blocks = [bf16_w] * 3 + [fp8_w] * 24
+    mergers = [{"fc1_w": None}] * 4
+    ov.tower_forward(np.zeros((4, 1152)), blocks, mergers, [(2, 2)])
+    assert calls == ["bf16"] * 3 + ["fp8"] * 24
