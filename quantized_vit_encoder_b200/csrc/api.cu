@@ -519,12 +519,14 @@ static int fill_grids(const int32_t* grid_hw, int n_images, bool need_even, Grid
     const int h = grid_hw[2 * i], w = grid_hw[2 * i + 1];
     VITQ_CHECK(h > 0 && w > 0, VITQ_ERR_INVALID_ARG);
     if (need_even) VITQ_CHECK(h % 2 == 0 && w % 2 == 0, VITQ_ERR_SHAPE);
+    const long long hw = (long long)h * w;   // 64-bit: h * w can exceed the int range
+    VITQ_CHECK(hw < (1ll << 30), VITQ_ERR_SHAPE);
     g->hw[2 * i] = h;
     g->hw[2 * i + 1] = w;
-    tot += (long long)h * w;
-    if (h * w > mx) mx = h * w;
+    tot += hw;
+    VITQ_CHECK(tot < (1ll << 30), VITQ_ERR_SHAPE);
+    if (hw > mx) mx = (int)hw;
   }
-  VITQ_CHECK(tot < (1ll << 30), VITQ_ERR_SHAPE);
   *n_total = (int)tot;
   *max_len = mx;
   return VITQ_OK;

@@ -63,3 +63,15 @@ def test_invalid_arguments_rejected_before_any_launch(built_lib):
     assert lib.vit_merger_forward(None, fake, 8, fake, fake, 1 << 30, None) == 1
     g = (ctypes.c_int32 * 2)(3, 4)
     assert lib.vit_positions(ctypes.cast(g, v), 0, fake, fake, None) == 1
+
+
+def test_oversized_grids_rejected_on_the_host(built_lib):
+    """Grid sizes whose patch count leaves the int range are a shape error, found before any launch."""
+    lib = built_lib
+    v = ctypes.c_void_p
+    fake = v(4096)
+    for hw in ((65536, 65536), (1 << 16, 1 << 15), (40000, 30000)):
+        g = (ctypes.c_int32 * 2)(*hw)
+        assert lib.vit_positions(ctypes.cast(g, v), 1, fake, fake, None) == 2
+    g = (ctypes.c_int32 * 4)(20000, 30000, 20000, 30000)      # each fits, the total does not
+    assert lib.vit_positions(ctypes.cast(g, v), 2, fake, fake, None) == 2
