@@ -62,6 +62,13 @@ typedef enum {
 #define VITQ_BLOCKS 27
 #define VITQ_MAX_IMAGES 64
 
+/* Size limits, checked on the host by every entry point (VITQ_ERR_SHAPE beyond
+ * them; the *_workspace_bytes functions return 0).  Within them every index the
+ * kernels form in 32-bit arithmetic (rows x 36 rotary items, rows x 32 lanes,
+ * tile counts, (M + 127) / 128) stays in the int range. */
+#define VITQ_MAX_ROWS (1 << 24) /* M, n_tokens, max_seqlen, and a tower's total patch count */
+#define VITQ_MAX_DIM (1 << 16)  /* N and K of the GEMM and quantisation primitives */
+
 /* Weights of one ViT block ([VE] ViTBlock): LayerNorm gamma/beta and biases are
  * bf16; each linear is FP8 codes [out, in] plus fp32 128x128 block scales. */
 typedef struct {

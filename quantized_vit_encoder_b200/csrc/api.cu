@@ -420,7 +420,7 @@ extern "C" {
 int vit_quant_act(const void* x, int M, int K, int ldx, uint8_t* q, float* s, int lds, void* stream) {
   VITQ_CHECK(x && q && s, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(M >= 0 && K > 0 && ldx >= K && lds >= M, VITQ_ERR_INVALID_ARG);
-  VITQ_CHECK(K % 16 == 0 && K <= 4608 && ldx % 8 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(K % 16 == 0 && K <= 4608 && ldx % 8 == 0 && M <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(x) && al16(q), VITQ_ERR_ALIGN);
   int r = current_device_ok(nullptr);
   if (r) return r;
@@ -431,7 +431,7 @@ int vit_quant_act(const void* x, int M, int K, int ldx, uint8_t* q, float* s, in
 int vit_quant_weight(const void* w, int N, int K, uint8_t* q, float* s, void* stream) {
   VITQ_CHECK(w && q && s, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(N >= 0 && K > 0, VITQ_ERR_INVALID_ARG);
-  VITQ_CHECK(K % 16 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(K % 16 == 0 && N <= VITQ_MAX_DIM && K <= VITQ_MAX_DIM, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(w) && al16(q), VITQ_ERR_ALIGN);
   int r = current_device_ok(nullptr);
   if (r) return r;
@@ -443,7 +443,7 @@ int vit_ln_quant(const void* x, int M, int K, int ldx, const void* gamma, const 
                  uint8_t* q, float* s, int lds, void* stream) {
   VITQ_CHECK(x && gamma && beta && q && s, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(M >= 0 && K > 0 && ldx >= K && lds >= M && eps >= 0.f, VITQ_ERR_INVALID_ARG);
-  VITQ_CHECK(K % 16 == 0 && K <= 4608 && ldx % 8 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(K % 16 == 0 && K <= 4608 && ldx % 8 == 0 && M <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(x) && al16(q) && al16(gamma) && al16(beta), VITQ_ERR_ALIGN);
   int r = current_device_ok(nullptr);
   if (r) return r;
@@ -455,7 +455,7 @@ int vit_ln_quant(const void* x, int M, int K, int ldx, const void* gamma, const 
 int vit_gelu_quant(const void* f, int M, int K, int ldf, uint8_t* q, float* s, int lds, void* stream) {
   VITQ_CHECK(f && q && s, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(M >= 0 && K > 0 && ldf >= K && lds >= M, VITQ_ERR_INVALID_ARG);
-  VITQ_CHECK(K % 16 == 0 && ldf % 8 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(K % 16 == 0 && ldf % 8 == 0 && M <= VITQ_MAX_ROWS && K <= VITQ_MAX_DIM, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(f) && al16(q), VITQ_ERR_ALIGN);
   int sms = 0;
   int r = current_device_ok(&sms);
@@ -470,6 +470,7 @@ int fp8_block_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W
   VITQ_CHECK(A && sA && W && sW && C, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(M >= 0 && N > 0 && K > 0 && ldsA >= M, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(K % 16 == 0 && N % 8 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(M <= VITQ_MAX_ROWS && N <= VITQ_MAX_DIM && K <= VITQ_MAX_DIM, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(A) && al16(W) && al16(C) && (!bias || al16(bias)) && (!residual || al16(residual)),
              VITQ_ERR_ALIGN);
   int sms = 0;
@@ -483,6 +484,7 @@ int bf16_gemm(const void* A, const void* W, const void* bias, const void* residu
   VITQ_CHECK(A && W && C, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(M >= 0 && N > 0 && K > 0, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(K % 8 == 0 && N % 8 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(M <= VITQ_MAX_ROWS && N <= VITQ_MAX_DIM && K <= VITQ_MAX_DIM, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(A) && al16(W) && al16(C) && (!bias || al16(bias)) && (!residual || al16(residual)),
              VITQ_ERR_ALIGN);
   int sms = 0;
@@ -494,6 +496,7 @@ int bf16_gemm(const void* A, const void* W, const void* bias, const void* residu
 
 int vit_rope_table(const int32_t* pos_hw, int n_tokens, float theta, float* cos_sin, void* stream) {
   VITQ_CHECK(pos_hw && cos_sin && n_tokens >= 0 && theta > 0.f, VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(n_tokens <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
   int r = current_device_ok(nullptr);
   if (r) return r;
   VITQ_LAUNCH("rope_table", S(stream), 0, (double)n_tokens * (8 + 288), launch_rope_table(pos_hw, n_tokens, (double)theta, cos_sin, S(stream)));
@@ -502,6 +505,7 @@ int vit_rope_table(const int32_t* pos_hw, int n_tokens, float theta, float* cos_
 
 int vit_rope2d(void* qkv, int n_tokens, const float* cos_sin, int flags, void* stream) {
   VITQ_CHECK(qkv && cos_sin && n_tokens >= 0 && (flags & ~VITQ_V_FP16) == 0, VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(n_tokens <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(qkv), VITQ_ERR_ALIGN);
   int r = current_device_ok(nullptr);
   if (r) return r;
@@ -520,11 +524,11 @@ static int fill_grids(const int32_t* grid_hw, int n_images, bool need_even, Grid
     VITQ_CHECK(h > 0 && w > 0, VITQ_ERR_INVALID_ARG);
     if (need_even) VITQ_CHECK(h % 2 == 0 && w % 2 == 0, VITQ_ERR_SHAPE);
     const long long hw = (long long)h * w;   // 64-bit: h * w can exceed the int range
-    VITQ_CHECK(hw < (1ll << 30), VITQ_ERR_SHAPE);
+    VITQ_CHECK(hw <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
     g->hw[2 * i] = h;
     g->hw[2 * i + 1] = w;
     tot += hw;
-    VITQ_CHECK(tot < (1ll << 30), VITQ_ERR_SHAPE);
+    VITQ_CHECK(tot <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
     if (hw > mx) mx = (int)hw;
   }
   *n_total = (int)tot;
@@ -548,7 +552,7 @@ int vit_attention_varlen(const void* qkv, int n_tokens, const int32_t* cu_seqlen
                          float softmax_scale, int flags, void* out, void* stream) {
   VITQ_CHECK(qkv && cu_seqlens && out && (flags & ~VITQ_V_FP16) == 0, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(n_tokens >= 0 && n_seqs >= 0 && max_seqlen >= 0 && softmax_scale > 0.f, VITQ_ERR_INVALID_ARG);
-  VITQ_CHECK(n_seqs <= 65535, VITQ_ERR_SHAPE);
+  VITQ_CHECK(n_seqs <= 65535 && n_tokens <= VITQ_MAX_ROWS && max_seqlen <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(qkv) && al16(out), VITQ_ERR_ALIGN);
   int r = current_device_ok(nullptr);
   if (r) return r;
@@ -558,21 +562,21 @@ int vit_attention_varlen(const void* qkv, int n_tokens, const int32_t* cu_seqlen
 }
 
 size_t vitq_block_workspace_bytes(int n_tokens) {
-  if (n_tokens < 0) return 0;
+  if (n_tokens < 0 || n_tokens > VITQ_MAX_ROWS) return 0;
   Carver c{nullptr};
   carve_block(c, n_tokens);
   return c.used;
 }
 
 size_t vitq_merger_workspace_bytes(int n_tokens) {
-  if (n_tokens < 0) return 0;
+  if (n_tokens < 0 || n_tokens > VITQ_MAX_ROWS) return 0;
   Carver c{nullptr};
   carve_merger(c, n_tokens);
   return c.used;
 }
 
 size_t vitq_tower_workspace_bytes(int n_tokens_max, int n_images_max) {
-  if (n_tokens_max < 0 || n_images_max < 1) return 0;
+  if (n_tokens_max < 0 || n_tokens_max > VITQ_MAX_ROWS || n_images_max < 1) return 0;
   Carver c{nullptr};
   carve_tower_head(c, n_tokens_max, n_images_max);
   Carver b{nullptr};
@@ -591,6 +595,7 @@ int vit_block_forward(const vitq_block_weights* w, void* x, int n_tokens, const 
   VITQ_CHECK(block_weights_ok(w), w ? VITQ_ERR_ALIGN : VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(x && cu_seqlens && cos_sin && ws, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(n_tokens >= 0 && n_seqs >= 0 && max_seqlen >= 0, VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(n_tokens <= VITQ_MAX_ROWS && max_seqlen <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(x) && al16(ws), VITQ_ERR_ALIGN);
   VITQ_CHECK(ws_bytes >= vitq_block_workspace_bytes(n_tokens), VITQ_ERR_WORKSPACE);
   int sms = 0;
@@ -606,7 +611,7 @@ int vit_merger_forward(const vitq_merger_weights* w, const void* x, int n_tokens
                        size_t ws_bytes, void* stream) {
   VITQ_CHECK(merger_weights_ok(w), w ? VITQ_ERR_ALIGN : VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(x && out && ws && n_tokens >= 0, VITQ_ERR_INVALID_ARG);
-  VITQ_CHECK(n_tokens % 4 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(n_tokens % 4 == 0 && n_tokens <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(x) && al16(out) && al16(ws), VITQ_ERR_ALIGN);
   VITQ_CHECK(ws_bytes >= vitq_merger_workspace_bytes(n_tokens), VITQ_ERR_WORKSPACE);
   int sms = 0;
@@ -715,6 +720,7 @@ int vit_block_forward_bf16(const vitq_block_weights_bf16* w, void* x, int n_toke
   VITQ_CHECK(block_bf16_weights_ok(w), w ? VITQ_ERR_ALIGN : VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(x && cu_seqlens && cos_sin && ws, VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(n_tokens >= 0 && n_seqs >= 0 && max_seqlen >= 0, VITQ_ERR_INVALID_ARG);
+  VITQ_CHECK(n_tokens <= VITQ_MAX_ROWS && max_seqlen <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(x) && al16(ws), VITQ_ERR_ALIGN);
   VITQ_CHECK(ws_bytes >= vitq_block_workspace_bytes(n_tokens), VITQ_ERR_WORKSPACE);
   int sms = 0;
@@ -728,7 +734,7 @@ int vit_block_forward_bf16(const vitq_block_weights_bf16* w, void* x, int n_toke
 }
 
 size_t vitq_patch_embed_workspace_bytes(int n_tokens) {
-  if (n_tokens < 0) return 0;
+  if (n_tokens < 0 || n_tokens > VITQ_MAX_ROWS) return 0;
   return up256((size_t)n_tokens * VITQ_HIDDEN * 2);
 }
 
@@ -755,7 +761,7 @@ int vit_patch_embed(const void* pixels, int n_tokens, const int32_t* grid_hw, in
 }
 
 size_t vitq_merger_bf16_workspace_bytes(int n_tokens) {
-  if (n_tokens < 0) return 0;
+  if (n_tokens < 0 || n_tokens > VITQ_MAX_ROWS) return 0;
   Carver c{nullptr};
   carve_merger_bf16(c, n_tokens);
   return c.used;
@@ -765,7 +771,7 @@ int vit_merger_forward_bf16(const vitq_merger_weights_bf16* w, const void* x, in
                             size_t ws_bytes, void* stream) {
   VITQ_CHECK(merger_bf16_weights_ok(w), w ? VITQ_ERR_ALIGN : VITQ_ERR_INVALID_ARG);
   VITQ_CHECK(x && out && ws && n_tokens >= 0, VITQ_ERR_INVALID_ARG);
-  VITQ_CHECK(n_tokens % 4 == 0, VITQ_ERR_SHAPE);
+  VITQ_CHECK(n_tokens % 4 == 0 && n_tokens <= VITQ_MAX_ROWS, VITQ_ERR_SHAPE);
   VITQ_CHECK(al16(x) && al16(out) && al16(ws), VITQ_ERR_ALIGN);
   VITQ_CHECK(ws_bytes >= vitq_merger_bf16_workspace_bytes(n_tokens), VITQ_ERR_WORKSPACE);
   int sms = 0;

@@ -73,5 +73,63 @@ def test_oversized_grids_rejected_on_the_host(built_lib):
     for hw in ((65536, 65536), (1 << 16, 1 << 15), (40000, 30000)):
         g = (ctypes.c_int32 * 2)(*hw)
         assert lib.vit_positions(ctypes.cast(g, v), 1, fake, fake, None) == 2
-    g = (ctypes.c_int32 * 4)(20000, 30000, 20000, 30000)      # each fits, the total does not
+    g = (ctypes.c_int32 * 4)(4096, 3000, 4096, 3000)      # each fits, the total does not
     assert lib.vit_positions(ctypes.cast(g, v), 2, fake, fake, None) == 2
+
+
+MAX_ROWS, MAX_DIM = 1 << 24, 1 << 16
+
+
+def test_header_size_limits_match():
+    src = open(HEADER).read()
+    assert re.search(r"#define VITQ_MAX_ROWS \(1 << 24\)", src)
+    assert re.search(r"#define VITQ_MAX_DIM \(1 << 16\)", src)
+
+
+def test_size_limits_rejected_on_the_host(built_lib):
+    """Counts past VITQ_MAX_ROWS / VITQ_MAX_DIM are a shape error at every entry point,
+    found before any device query (so the status comes back here, without a GPU), and
+    the workspace sizes are 0 past the limit but not at it."""
+    lib = built_lib
+    v, i = ctypes.c_void_p, ctypes.c_int
+    fake = v(4096)
+    R, D = MAX_ROWS + 1, MAX_DIM + 8
+    assert lib.vit_quant_act(fake, R, 128, 128, fake, fake, R, None) == 2
+    assert lib.vit_ln_quant(fake, R, 128, 128, fake, fake, ctypes.c_float(1e-6), fake, fake, R, None) == 2
+    assert lib.vit_gelu_quant(fake, R, 128, 128, fake, fake, R, None) == 2
+    assert lib.vit_gelu_quant(fake, 8, MAX_DIM + 16, MAX_DIM + 16, fake, fake, 8, None) == 2
+    assert lib.vit_quant_weight(fake, D, 128, fake, fake, None) == 2
+    assert lib.vit_quant_weight(fake, 128, MAX_DIM + 16, fake, fake, None) == 2
+    # M near the int maximum: (M + 127) / 128 must never be formed
+    for m, n, k in ((R, 64, 128), ((1 << 31) - 1, 64, 128), (8, D, 128), (8, 64, MAX_DIM + 16)):
+        assert lib.fp8_block_gemm(fake, fake, m, fake, fake, None, None, fake, m, n, k, None) == 2
+        assert lib.bf16_gemm(fake, fake, None, None, fake, m, n, k, None) == 2
+    assert lib.vit_rope_table(fake, R, ctypes.c_float(10000.0), fake, None) == 2
+    assert lib.vit_rope2d(fake, R, fake, 0, None) == 2
+    assert lib.vit_attention_varlen(fake, R, fake, 1, 16, ctypes.c_float(0.1), 0, fake, None) == 2
+    assert lib.vit_attention_varlen(fake, 16, fake, 1, R, ctypes.c_float(0.1), 0, fake, None) == 2
+
+    from quantized_vit_encoder_b200 import vitq
+    bw = vitq.BlockWeights(*([4096] * len(vitq.BlockWeights._fields_)))
+    mw = vitq.MergerWeights(*([4096] * len(vitq.MergerWeights._fields_)))
+    bw16 = vitq.BlockWeightsBf16(*([4096] * len(vitq.BlockWeightsBf16._fields_)))
+    mw16 = vitq.MergerWeightsBf16(*([4096] * len(vitq.MergerWeightsBf16._fields_)))
+    big = ctypes.c_size_t(1 << 62)
+    ref = ctypes.byref
+    assert lib.vit_block_forward(ref(bw), fake, R, fake, 1, 16, fake, fake, big, None) == 2
+    assert lib.vit_block_forward(ref(bw), fake, 16, fake, 1, R, fake, fake, big, None) == 2
+    assert lib.vit_block_forward_bf16(ref(bw16), fake, R, fake, 1, 16, fake, fake, big, None) == 2
+    assert lib.vit_merger_forward(ref(mw), fake, MAX_ROWS + 4, fake, fake, big, None) == 2
+    assert lib.vit_merger_forward_bf16(ref(mw16), fake, MAX_ROWS + 4, fake, fake, big, None) == 2
+    g = (ctypes.c_int32 * 2)(4096, 4098)                      # 16785408 patches, one image
+    assert lib.vit_patch_embed(fake, 4096 * 4098, ctypes.cast(g, v), 1, fake, fake, fake, fake, fake, big,
+                               None) == 2
+
+    for name in ("vitq_block_workspace_bytes", "vitq_merger_workspace_bytes",
+                 "vitq_patch_embed_workspace_bytes", "vitq_merger_bf16_workspace_bytes"):
+        f = getattr(lib, name)
+        f.restype, f.argtypes = ctypes.c_size_t, [i]
+        assert f(MAX_ROWS) > 0 and f(MAX_ROWS + 4) == 0 and f(-4) == 0, name
+    f = lib.vitq_tower_workspace_bytes
+    f.restype, f.argtypes = ctypes.c_size_t, [i, i]
+    assert f(MAX_ROWS, 4) > 0 and f(MAX_ROWS + 4, 4) == 0
