@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libvitq.so")
 
 HIDDEN, HEADS, HEAD_DIM, MLP, QKV = 1152, 16, 72, 4304, 3456
 MERGE_IN, OUT_HIDDEN, N_BLOCKS = 4608, 2048, 27
+PATCH_DIM, POS_GRID = 1536, 48
 STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "pointer not 16-byte aligned",
           4: "device is not sm_100", 5: "CUDA error", 6: "workspace too small",
           7: "device pipeline wait timed out"}
@@ -127,6 +128,47 @@ def _p(t):
     return None if t is None else C.c_void_p(t.data_ptr())
 
 
+_DEVICE_TYPE = "cuda"
+_bf16, _f32, _u8, _i32 = torch.bfloat16, torch.float32, torch.uint8, torch.int32
+
+
+def _arg(t, name, dtype, shape=None, rows=False):
+    """Check a tensor before its pointer crosses the ABI: device memory, the dtype
+    the C side reads, the shape (None entries are free) and a dense layout
+    (rows=True: each row dense, the row stride is passed to the C side)."""
+    if not isinstance(t, torch.Tensor):
+        raise VitqError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if t.device.type != _DEVICE_TYPE:
+        raise VitqError(f"{name}: tensor on {t.device}; the library reads device memory only")
+    if t.dtype != dtype:
+        raise VitqError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if shape is not None and (t.dim() != len(shape) or
+                              any(w is not None and w != d for w, d in zip(shape, t.shape))):
+        raise VitqError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    dense = (t.dim() == 2 and t.stride(1) == 1 and t.stride(0) >= t.shape[1]) if rows else t.is_contiguous()
+    if not dense:
+        raise VitqError(f"{name}: strides {t.stride()} are not a dense{' row' if rows else ''} layout")
+    return t
+
+
+def _cs(cos_sin, n):
+    _arg(cos_sin, "cos_sin", _f32, (None, 72))
+    if cos_sin.shape[0] < n:
+        raise VitqError(f"cos_sin: {cos_sin.shape[0]} rows for {n} tokens")
+    return cos_sin
+
+
+def _cu(cu_seqlens):
+    _arg(cu_seqlens, "cu_seqlens", _i32, (None,))
+    if cu_seqlens.shape[0] < 1:
+        raise VitqError("cu_seqlens: needs at least one entry")
+    return cu_seqlens
+
+
+def _ws(ws):
+    return _arg(ws, "ws", _u8, (None,))
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return C.c_void_p(s.cuda_stream)
@@ -171,7 +213,7 @@ def _scales(nkb, M, device):
 
 def quant_act(x: torch.Tensor, stream=None):
     """1x128 FP8 quantisation of bf16 x [M, K] -> (codes uint8 [M, K], scales fp32 [ceil(K/128), M_pad4])."""
-    M, K = x.shape
+    M, K = _arg(x, "x", _bf16, (None, None), rows=True).shape
     q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
     s, lds = _scales((K + 127) // 128, M, x.device)
     _check(load().vit_quant_act(_p(x), M, K, x.stride(0), _p(q), _p(s), lds, _stream(stream)), "vit_quant_act")
@@ -180,7 +222,7 @@ def quant_act(x: torch.Tensor, stream=None):
 
 def quant_weight(w: torch.Tensor, stream=None):
     """128x128-block FP8 quantisation of bf16 w [N, K] -> (codes [N, K], scales [ceil(N/128), ceil(K/128)])."""
-    N, K = w.shape
+    N, K = _arg(w, "w", _bf16, (None, None)).shape
     q = torch.empty((N, K), dtype=torch.uint8, device=w.device)
     s = torch.zeros(((N + 127) // 128, (K + 127) // 128), dtype=torch.float32, device=w.device)
     _check(load().vit_quant_weight(_p(w), N, K, _p(q), _p(s), _stream(stream)), "vit_quant_weight")
@@ -188,7 +230,9 @@ def quant_weight(w: torch.Tensor, stream=None):
 
 
 def ln_quant(x, gamma, beta, eps: float = 1e-6, stream=None):
-    M, K = x.shape
+    M, K = _arg(x, "x", _bf16, (None, None), rows=True).shape
+    _arg(gamma, "gamma", _bf16, (K,))
+    _arg(beta, "beta", _bf16, (K,))
     q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
     s, lds = _scales((K + 127) // 128, M, x.device)
     _check(load().vit_ln_quant(_p(x), M, K, x.stride(0), _p(gamma), _p(beta), eps, _p(q), _p(s), lds,
@@ -197,7 +241,7 @@ def ln_quant(x, gamma, beta, eps: float = 1e-6, stream=None):
 
 
 def gelu_quant(f, stream=None):
-    M, K = f.shape
+    M, K = _arg(f, "f", _bf16, (None, None), rows=True).shape
     q = torch.empty((M, K), dtype=torch.uint8, device=f.device)
     s, lds = _scales((K + 127) // 128, M, f.device)
     _check(load().vit_gelu_quant(_p(f), M, K, f.stride(0), _p(q), _p(s), lds, _stream(stream)), "vit_gelu_quant")
@@ -206,8 +250,18 @@ def gelu_quant(f, stream=None):
 
 def fp8_block_gemm(qa, sa, qw, sw, bias=None, residual=None, out=None, stream=None):
     """bf16 C [M, N] = block-scaled FP8 product (+ bias) (+ residual)."""
-    M, K = qa.shape
-    N = qw.shape[0]
+    M, K = _arg(qa, "qa", _u8, (None, None)).shape
+    N = _arg(qw, "qw", _u8, (None, K)).shape[0]
+    _arg(sa, "sa", _f32, ((K + 127) // 128, None), rows=True)
+    if sa.shape[1] < M:
+        raise VitqError(f"sa: {sa.shape[1]} columns for {M} rows")
+    _arg(sw, "sw", _f32, ((N + 127) // 128, (K + 127) // 128))
+    if bias is not None:
+        _arg(bias, "bias", _bf16, (N,))
+    if residual is not None:
+        _arg(residual, "residual", _bf16, (M, N))
+    if out is not None:
+        _arg(out, "out", _bf16, (M, N))
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=qa.device)
     _check(load().fp8_block_gemm(_p(qa), _p(sa), sa.stride(0), _p(qw), _p(sw), _p(bias), _p(residual), _p(out),
@@ -217,8 +271,14 @@ def fp8_block_gemm(qa, sa, qw, sw, bias=None, residual=None, out=None, stream=No
 
 def bf16_gemm(a, w, bias=None, residual=None, out=None, stream=None):
     """bf16 C [M, N] = a [M, K] w[N, K]^T (+ bias) (+ residual), fp32 accumulation."""
-    M, K = a.shape
-    N = w.shape[0]
+    M, K = _arg(a, "a", _bf16, (None, None)).shape
+    N = _arg(w, "w", _bf16, (None, K)).shape[0]
+    if bias is not None:
+        _arg(bias, "bias", _bf16, (N,))
+    if residual is not None:
+        _arg(residual, "residual", _bf16, (M, N))
+    if out is not None:
+        _arg(out, "out", _bf16, (M, N))
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     _check(load().bf16_gemm(_p(a), _p(w), _p(bias), _p(residual), _p(out), M, N, K, _stream(stream)), "bf16_gemm")
@@ -226,7 +286,7 @@ def bf16_gemm(a, w, bias=None, residual=None, out=None, stream=None):
 
 
 def rope_table(pos_hw: torch.Tensor, theta: float = 10000.0, stream=None):
-    n = pos_hw.shape[0]
+    n = _arg(pos_hw, "pos_hw", _i32, (None, 2)).shape[0]
     cs = torch.empty((n, 72), dtype=torch.float32, device=pos_hw.device)
     _check(load().vit_rope_table(_p(pos_hw), n, theta, _p(cs), _stream(stream)), "vit_rope_table")
     return cs
@@ -237,6 +297,7 @@ V_FP16 = 1
 
 def rope2d_(qkv: torch.Tensor, cos_sin: torch.Tensor, flags: int = 0, stream=None):
     """In-place 2D rotary on the q, k parts of qkv; flags=V_FP16 also converts v to fp16 in place."""
+    _cs(cos_sin, _arg(qkv, "qkv", _bf16, (None, QKV)).shape[0])
     _check(load().vit_rope2d(_p(qkv), qkv.shape[0], _p(cos_sin), flags, _stream(stream)), "vit_rope2d")
     return qkv
 
@@ -254,9 +315,11 @@ def positions(grids, device="cuda", stream=None):
 
 def attention_varlen(qkv, cu_seqlens, max_seqlen: int, scale: float | None = None, out=None, flags: int = 0,
                      stream=None):
-    n = qkv.shape[0]
+    n = _arg(qkv, "qkv", _bf16, (None, QKV)).shape[0]
+    _cu(cu_seqlens)
     if out is None:
         out = torch.empty((n, HIDDEN), dtype=torch.bfloat16, device=qkv.device)
+    _arg(out, "out", _bf16, (n, HIDDEN))
     if scale is None:
         scale = 1.0 / math.sqrt(HEAD_DIM)
     _check(load().vit_attention_varlen(_p(qkv), n, _p(cu_seqlens), cu_seqlens.shape[0] - 1, max_seqlen, scale,
@@ -266,11 +329,45 @@ def attention_varlen(qkv, cu_seqlens, max_seqlen: int, scale: float | None = Non
 
 # ---------------------------------------------------------------- layers
 
+BLOCK_SHAPES = {"norm1_w": (HIDDEN,), "norm1_b": (HIDDEN,), "qkv_w": (QKV, HIDDEN), "qkv_b": (QKV,),
+                "proj_w": (HIDDEN, HIDDEN), "proj_b": (HIDDEN,), "norm2_w": (HIDDEN,), "norm2_b": (HIDDEN,),
+                "fc1_w": (MLP, HIDDEN), "fc1_b": (MLP,), "fc2_w": (HIDDEN, MLP), "fc2_b": (HIDDEN,)}
+MERGER_SHAPES = {"norm_w": (MERGE_IN,), "norm_b": (MERGE_IN,), "fc1_w": (MERGE_IN, MERGE_IN),
+                 "fc1_b": (MERGE_IN,), "fc2_w": (OUT_HIDDEN, MERGE_IN), "fc2_b": (OUT_HIDDEN,)}
+
+
+def _weights(params: dict, shapes: dict, device) -> dict:
+    """The bf16 weights a block or merger needs, on the device, dense, shape-checked."""
+    missing = [k for k in shapes if k not in params]
+    if missing:
+        raise VitqError(f"weights missing: {missing}")
+    t = {k: params[k].to(device).contiguous() for k in shapes}
+    for k, shp in shapes.items():
+        _arg(t[k], k, _bf16, shp)
+    return t
+
+
+def _x(x, name="x"):
+    return _arg(x, name, _bf16, (None, HIDDEN)).shape[0]
+
+
+def _merged_out(out, n, name="out"):
+    if n % 4:
+        raise VitqError(f"{n} tokens: the 2x2 merger takes a multiple of 4")
+    return _arg(out, name, _bf16, (n // 4, OUT_HIDDEN))
+
+
+def _taps(taps, n):
+    if len(taps) != 4:
+        raise VitqError(f"taps: {len(taps)} tensors, the tower has 4 mergers")
+    for i, t in enumerate(taps):
+        _merged_out(t, n, f"taps[{i}]")
+
 class DeviceBlock:
     """Device-resident block weights (bf16 vectors, FP8 codes, fp32 scales) and their C struct."""
 
     def __init__(self, params: dict, device="cuda", stream=None):
-        t = {k: v.to(device) for k, v in params.items()}
+        t = _weights(params, BLOCK_SHAPES, device)
         self.t = t
         for name in ("qkv", "proj", "fc1", "fc2"):
             t[name + "_q"], t[name + "_s"] = quant_weight(t[name + "_w"], stream)
@@ -279,7 +376,7 @@ class DeviceBlock:
 
 class DeviceMerger:
     def __init__(self, params: dict, device="cuda", stream=None):
-        t = {k: v.to(device) for k, v in params.items()}
+        t = _weights(params, MERGER_SHAPES, device)
         self.t = t
         for name in ("fc1", "fc2"):
             t[name + "_q"], t[name + "_s"] = quant_weight(t[name + "_w"], stream)
@@ -290,13 +387,13 @@ class DeviceBlockBf16:
     """Device-resident bf16 block weights (no quantisation) and their C struct."""
 
     def __init__(self, params: dict, device="cuda"):
-        self.t = {k: v.to(device).contiguous() for k, v in params.items()}
+        self.t = _weights(params, BLOCK_SHAPES, device)
         self.struct = BlockWeightsBf16(**{f: self.t[f].data_ptr() for f, _ in BlockWeightsBf16._fields_})
 
 
 class DeviceMergerBf16:
     def __init__(self, params: dict, device="cuda"):
-        self.t = {k: v.to(device).contiguous() for k, v in params.items()}
+        self.t = _weights(params, MERGER_SHAPES, device)
         self.struct = MergerWeightsBf16(**{f: self.t[f].data_ptr() for f, _ in MergerWeightsBf16._fields_})
 
 
@@ -316,6 +413,9 @@ class DeviceTowerMixed:
 
 def block_forward_bf16_(blk: DeviceBlockBf16, x, cu_seqlens, max_seqlen, cos_sin, ws, stream=None):
     """In-place bf16 block forward on bf16 x [n, 1152]."""
+    _cs(cos_sin, _x(x))
+    _cu(cu_seqlens)
+    _ws(ws)
     _check(load().vit_block_forward_bf16(C.byref(blk.struct), _p(x), x.shape[0], _p(cu_seqlens),
                                          cu_seqlens.shape[0] - 1, max_seqlen, _p(cos_sin), _p(ws), ws.numel(),
                                          _stream(stream)), "vit_block_forward_bf16")
@@ -327,9 +427,11 @@ def merger_bf16_workspace_bytes(n: int) -> int:
 
 
 def merger_forward_bf16(mg: DeviceMergerBf16, x, ws, out=None, stream=None):
-    n = x.shape[0]
+    n = _x(x)
+    _ws(ws)
     if out is None:
         out = torch.empty((n // 4, OUT_HIDDEN), dtype=torch.bfloat16, device=x.device)
+    _merged_out(out, n)
     _check(load().vit_merger_forward_bf16(C.byref(mg.struct), _p(x), n, _p(out), _p(ws), ws.numel(),
                                           _stream(stream)), "vit_merger_forward_bf16")
     return out
@@ -337,9 +439,11 @@ def merger_forward_bf16(mg: DeviceMergerBf16, x, ws, out=None, stream=None):
 
 def tower_forward_mixed_(tower: DeviceTowerMixed, x, grids, ws, taps=None, stream=None):
     """In-place mixed-precision tower forward; returns the four taps [n/4, 2048]."""
-    n = x.shape[0]
+    n = _x(x)
+    _ws(ws)
     if taps is None:
         taps = [torch.empty((n // 4, OUT_HIDDEN), dtype=torch.bfloat16, device=x.device) for _ in range(4)]
+    _taps(taps, n)
     g = (C.c_int32 * (2 * len(grids)))(*[v for hw in grids for v in hw])
     tp = (C.c_void_p * 4)(*[t.data_ptr() for t in taps])
     _check(load().vit_tower_forward_mixed(C.byref(tower.struct), _p(x), C.cast(g, C.c_void_p), len(grids), tp,
@@ -349,11 +453,16 @@ def tower_forward_mixed_(tower: DeviceTowerMixed, x, grids, ws, taps=None, strea
 
 def patch_embed(pixels, grids, w, b, pos_table, out=None, ws=None, stream=None):
     """bf16 x [n, 1152] = pixels [n, 1536] . w^T + b + interpolated position embedding."""
-    n = pixels.shape[0]
+    n = _arg(pixels, "pixels", _bf16, (None, PATCH_DIM)).shape[0]
+    _arg(w, "w", _bf16, (HIDDEN, PATCH_DIM))
+    _arg(b, "b", _bf16, (HIDDEN,))
+    _arg(pos_table, "pos_table", _bf16, (POS_GRID * POS_GRID, HIDDEN))
     if out is None:
         out = torch.empty((n, HIDDEN), dtype=torch.bfloat16, device=pixels.device)
+    _arg(out, "out", _bf16, (n, HIDDEN))
     if ws is None:
         ws = workspace(int(load().vitq_patch_embed_workspace_bytes(n)), pixels.device)
+    _ws(ws)
     g = (C.c_int32 * (2 * len(grids)))(*[v for hw in grids for v in hw])
     _check(load().vit_patch_embed(_p(pixels), n, C.cast(g, C.c_void_p), len(grids), _p(w), _p(b), _p(pos_table),
                                   _p(out), _p(ws), ws.numel(), _stream(stream)), "vit_patch_embed")
@@ -378,6 +487,9 @@ def workspace(nbytes: int, device="cuda"):
 
 def block_forward_(blk: DeviceBlock, x, cu_seqlens, max_seqlen, cos_sin, ws, stream=None):
     """In-place block forward on bf16 x [n, 1152]."""
+    _cs(cos_sin, _x(x))
+    _cu(cu_seqlens)
+    _ws(ws)
     _check(load().vit_block_forward(C.byref(blk.struct), _p(x), x.shape[0], _p(cu_seqlens), cu_seqlens.shape[0] - 1,
                                     max_seqlen, _p(cos_sin), _p(ws), ws.numel(), _stream(stream)),
            "vit_block_forward")
@@ -385,9 +497,11 @@ def block_forward_(blk: DeviceBlock, x, cu_seqlens, max_seqlen, cos_sin, ws, str
 
 
 def merger_forward(mg: DeviceMerger, x, ws, out=None, stream=None):
-    n = x.shape[0]
+    n = _x(x)
+    _ws(ws)
     if out is None:
         out = torch.empty((n // 4, OUT_HIDDEN), dtype=torch.bfloat16, device=x.device)
+    _merged_out(out, n)
     _check(load().vit_merger_forward(C.byref(mg.struct), _p(x), n, _p(out), _p(ws), ws.numel(), _stream(stream)),
            "vit_merger_forward")
     return out
@@ -399,6 +513,7 @@ MERGER_STATIC_MAX_TOKENS = 4096
 def merger_forward_static(mg: DeviceMerger, x, out):
     """vit_merger_forward_static: the merger with the library's fixed scratch
     (no workspace, no allocation); out must be given, bf16 [n/4, 2048]."""
+    _merged_out(out, _x(x))
     _check(load().vit_merger_forward_static(C.byref(mg.struct), _p(x), x.shape[0], _p(out), _stream(None)),
            "vit_merger_forward_static")
     return out
@@ -416,9 +531,11 @@ class DeviceTower:
 
 def tower_forward_(tower: DeviceTower, x, grids, ws, taps=None, stream=None):
     """In-place tower forward on bf16 x [n, 1152]; returns the four tap tensors [n/4, 2048]."""
-    n = x.shape[0]
+    n = _x(x)
+    _ws(ws)
     if taps is None:
         taps = [torch.empty((n // 4, OUT_HIDDEN), dtype=torch.bfloat16, device=x.device) for _ in range(4)]
+    _taps(taps, n)
     g = (C.c_int32 * (2 * len(grids)))(*[v for hw in grids for v in hw])
     tp = (C.c_void_p * 4)(*[t.data_ptr() for t in taps])
     _check(load().vit_tower_forward(C.byref(tower.struct), _p(x), C.cast(g, C.c_void_p), len(grids), tp, _p(ws),
