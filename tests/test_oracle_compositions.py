@@ -9,7 +9,11 @@ oracle wires them together to facts that hold for the method itself:
 * with such blocks the tower state after block b follows that recursion, so the
   mergers must see the states after blocks 8, 16, 24 and 27 (1-indexed);
 * a block over packed images equals the block over each image alone, bit for bit
-  (every stage is row-wise except attention, which is per segment).
+  (every stage is row-wise except attention, which is per segment);
+* the 2x2 merger (FP8 and bf16) normalises the four concatenated rows as one 4608
+  row (constant rows give the closed-form values, not the zeros a per-row
+  LayerNorm would), maps rows 4i..4i+3 to output row i and nothing else, and ends
+  in fc2 with no residual (zero fc2 weights leave exactly its bias).
 """
 import numpy as np
 import pytest
@@ -119,3 +123,71 @@ def test_mixed_tower_runs_bf16_then_fp8_blocks(monkeypatch):
     mergers = [{"fc1_w": None}] * 4
     ov.tower_forward(np.zeros((4, 1152)), blocks, mergers, [(2, 2)])
     assert calls == ["bf16"] * 3 + ["fp8"] * 24
+
+
+# ---------------------------------------------------------------- the 2x2 merger
+
+def _merger_weights(seed, fp8=True, **override):
+    p = {k: _f64(v) for k, v in wl.merger_params(seed).items()}
+    p.update(override)
+    return ov.quantize_merger_weights(p) if fp8 else p
+
+
+def _merger(fp8):
+    return ov.merger_forward if fp8 else ov.merger_forward_bf16
+
+
+def _bf16_of(v):
+    """bf16 rounding by torch's cast (independent of the oracle's own rounding)."""
+    return torch.tensor(v, dtype=torch.float64).to(torch.bfloat16).double().numpy()
+
+
+@pytest.mark.parametrize("fp8", [True, False], ids=["fp8", "bf16"])
+def test_merger_layernorm_spans_the_four_concatenated_rows(fp8):
+    """Four constant rows c_j make one 4608 row whose LayerNorm (gamma 1, beta 0) is
+    (c_j - mean) / sqrt(var + eps) on features [1152 j, 1152 (j + 1)): nonzero, where a
+    LayerNorm over each 1152 row alone would give zeros, and in the row order."""
+    w = _merger_weights(61, fp8, norm_w=np.ones(4608), norm_b=np.zeros(4608))
+    groups = [(-3.0, -1.0, 1.0, 3.0), (2.0, 2.0, 2.0, 6.0)]
+    x = np.repeat(np.array(groups).reshape(8, 1), 1152, axis=1)
+    _, st = _merger(fp8)(x, w, keep=True)
+    for g, c in enumerate(groups):
+        c = np.array(c)
+        v = _bf16_of((c - c.mean()) / np.sqrt(((c - c.mean()) ** 2).mean() + 1e-6))
+        if not fp8:
+            assert np.array_equal(st["h1"][g], np.repeat(v, 1152))
+            continue
+        # each 128-column block lies inside one source row, so it is constant: codes +-448
+        # and scale fl32(|v_j| / 448)
+        blocks = np.repeat(v, 9)
+        want_s = (np.abs(blocks).astype(np.float32) / np.float32(448.0)).astype(np.float32)
+        assert np.array_equal(st["s1"][:, g], want_s)
+        want_q = np.repeat(np.where(blocks > 0, 0x7E, 0xFE), 128).astype(np.uint8)
+        assert np.array_equal(st["q1"][g], want_q)
+
+
+@pytest.mark.parametrize("fp8", [True, False], ids=["fp8", "bf16"])
+def test_merger_output_row_depends_on_its_four_rows_only(fp8):
+    """Output row i is a function of input rows 4i..4i+3: permuting the groups permutes
+    the output rows bit for bit, and changing one input row changes one output row."""
+    w = _merger_weights(62, fp8)
+    x = _f64(wl.random_bf16((16, 1152), 63, 1.0))
+    run = _merger(fp8)
+    out = run(x, w)
+    perm = [2, 0, 3, 1]
+    xp = np.concatenate([x[4 * g:4 * g + 4] for g in perm])
+    assert np.array_equal(run(xp, w), out[perm])
+    x2 = x.copy()
+    x2[5] = _f64(wl.random_bf16((1, 1152), 64, 1.0))[0]
+    out2 = run(x2, w)
+    changed = [i for i in range(4) if not np.array_equal(out2[i], out[i])]
+    assert changed == [1]
+
+
+@pytest.mark.parametrize("fp8", [True, False], ids=["fp8", "bf16"])
+def test_merger_with_zero_fc2_is_its_output_bias(fp8):
+    """fc2 is the last step and has no residual: zero fc2 weights leave b_fc2 on every row."""
+    w = _merger_weights(65, fp8, fc2_w=np.zeros((2048, 4608)))
+    x = _f64(wl.random_bf16((8, 1152), 66, 1.0))
+    out = _merger(fp8)(x, w)
+    assert np.array_equal(out, np.broadcast_to(w["fc2_b"], (2, 2048)))
