@@ -195,7 +195,11 @@ int vit_positions(const int32_t* grid_hw, int n_images, int32_t* pos_hw, int32_t
 /* Block-diagonal non-causal attention ([FRT] s1/s3 "FA2 (full, bidirectional)",
  * s5 cu_seqlens).  qkv: bf16 [n_tokens, 3, 16, 72] (rotary already applied);
  * cu_seqlens int32 [n_seqs + 1] with cu[0] = 0, cu[n_seqs] = n_tokens;
- * max_seqlen >= every segment length.  out: bf16 [n_tokens, 1152], head h in
+ * max_seqlen >= every segment length.  cu_seqlens lives in device memory and
+ * is read only by the kernel, so the host cannot check it: it must be
+ * non-decreasing from 0 (rows past n_tokens are neither read nor written;
+ * query rows of a segment past max_seqlen are left unwritten).  out: bf16
+ * [n_tokens, 1152], head h in
  * columns h*72 .. h*72+71.  qkv must be 16-byte aligned.  flags: 0 = v is bf16
  * and P is rounded to bf16 for P.V (flash-attention bf16 numerics);
  * VITQ_V_FP16 = v is fp16 (see vit_rope2d) and P is rounded to fp16. */
@@ -224,7 +228,9 @@ size_t vitq_patch_embed_workspace_bytes(int n_tokens);
 /* One ViT block in place on x bf16 [n_tokens, 1152] ([FRT] s3 per-block chain):
  * LN1+quant -> QKV GEMM+bias -> RoPE -> attention -> quant -> proj GEMM+bias+x
  * -> LN2+quant -> fc1 GEMM+bias -> GELU+quant -> fc2 GEMM+bias+residual.
- * cos_sin from vit_rope_table; ws >= vitq_block_workspace_bytes(n_tokens). */
+ * cu_seqlens, n_seqs, max_seqlen as for vit_attention_varlen (device memory,
+ * not checked by the host); cos_sin from vit_rope_table, fp32 [n_tokens, 72];
+ * ws >= vitq_block_workspace_bytes(n_tokens). */
 int vit_block_forward(const vitq_block_weights* w, void* x, int n_tokens, const int32_t* cu_seqlens,
                       int n_seqs, int max_seqlen, const float* cos_sin, void* ws, size_t ws_bytes,
                       void* stream);
