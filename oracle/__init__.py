@@ -17,10 +17,13 @@ vit      : the stages of the block (LayerNorm+quant, FP8 block-128 GEMM,
            2D rotary, varlen attention, GELU+quant), the 2x2 merger and the
            27-block tower with its DeepStack taps.
 
-Pinning: every function is checked against something other than itself in
-``tests/test_oracle_pins.py`` (closed forms, exhaustive code tables, library
-casts, brute-force loops, invariants).  The whole-block and whole-tower
-compositions have no published values to pin against ("parity unpinned"
-beyond their pinned stages).
+Pinning: every stage function is checked against something other than itself
+in ``tests/test_oracle_pins.py`` (closed forms, exhaustive code tables, library
+casts, brute-force loops, invariants).  The block, merger and tower have no
+published values; their wiring is pinned in ``tests/test_oracle_compositions.py``
+by closed forms and invariants of the method (zero-weight blocks reduce to their
+residual adds, the taps follow blocks 8, 16, 24 and 27, packed images equal
+images alone, the merger normalises four concatenated rows and maps each group
+of four rows to one output row), and their arithmetic through the pinned stages.
 """
 from . import numerics, vit  # noqa: F401
