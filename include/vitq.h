@@ -308,7 +308,8 @@ unsigned long long vitq_launch_count(void);
 /* Launch timing.  Between vitq_profile_start and vitq_profile_stop every kernel
  * launch of this library is bracketed by a CUDA event pair on its stream (not
  * for use during stream capture).  vitq_profile_stop waits for the events and
- * returns the number of records; vitq_profile_get returns record i: the kernel
+ * returns the number of records (-VITQ_ERR_CUDA if an event cannot be read);
+ * vitq_profile_get returns record i (VITQ_ERR_INVALID_ARG past the last): the kernel
  * name (static string), its device time in ms, and its algorithmic FLOPs and
  * HBM bytes (0 where the host does not know them). */
 void vitq_profile_start(void);

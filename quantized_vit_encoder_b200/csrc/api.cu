@@ -837,8 +837,9 @@ int vitq_profile_stop(void) {
   g_prof_on = false;
   g_prof_ms.assign(g_prof.size(), 0.f);
   for (size_t i = 0; i < g_prof.size(); ++i) {
-    if (cudaEventSynchronize(g_prof[i].b) != cudaSuccess) return VITQ_ERR_CUDA;
-    if (cudaEventElapsedTime(&g_prof_ms[i], g_prof[i].a, g_prof[i].b) != cudaSuccess) return VITQ_ERR_CUDA;
+    // negative on failure, so that an error is never read as a record count
+    if (cudaEventSynchronize(g_prof[i].b) != cudaSuccess) return -VITQ_ERR_CUDA;
+    if (cudaEventElapsedTime(&g_prof_ms[i], g_prof[i].a, g_prof[i].b) != cudaSuccess) return -VITQ_ERR_CUDA;
   }
   return (int)g_prof.size();
 }

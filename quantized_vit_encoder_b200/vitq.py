@@ -191,7 +191,7 @@ def profile_stop() -> list:
     lib = load()
     n = lib.vitq_profile_stop()
     if n < 0:
-        raise VitqError(f"vitq_profile_stop: {n}")
+        _check(-n, "vitq_profile_stop")
     out = []
     name, ms, fl, by = C.c_char_p(), C.c_float(), C.c_double(), C.c_double()
     for i in range(n):

@@ -50,6 +50,12 @@ def test_host_only_calls(built_lib):
     # codes (4304/row) + scales + qkv + attn + x1 + fc1 out, all bf16 or bytes
     assert b >= 6256 * (4304 + 2 * (3456 + 1152 + 1152 + 4304))
     assert lib.vitq_tower_workspace_bytes(9164, 4) > lib.vitq_block_workspace_bytes(9164)
+    # an empty profile needs no device: 0 records, and record 0 does not exist
+    lib.vitq_profile_start()
+    assert lib.vitq_profile_stop() == 0
+    name, ms, fl, by = ctypes.c_char_p(), ctypes.c_float(), ctypes.c_double(), ctypes.c_double()
+    ref = ctypes.byref
+    assert lib.vitq_profile_get(0, ref(name), ref(ms), ref(fl), ref(by)) == 1
 
 
 def test_invalid_arguments_rejected_before_any_launch(built_lib):
