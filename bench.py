@@ -190,6 +190,10 @@ def kernel_table(records, by_shape: bool = False) -> dict:
     return out
 
 
+# Public dense datasheet peaks of one B200 (context beside the measured denominators).
+NOMINAL = {"bf16": 2250.0, "fp8": 4500.0, "hbm_gbs": 7700.0}
+
+
 def roofline(table: dict, peaks: dict) -> dict:
     name, e = max(table.items(), key=lambda kv: kv[1]["ms"])
     per_launch_ms = e["ms"] / e["launches"]
@@ -207,8 +211,13 @@ def roofline(table: dict, peaks: dict) -> dict:
         t = json.load(open(tfile)).get(name)
         if t and t.get("source_sha") == _source_sha(t.get("source", "")):
             traffic = t.get("bytes_per_launch")
+    if bound == "tensor":
+        nominal = NOMINAL["fp8" if name == "fp8_block_gemm" else "bf16"]
+    else:
+        nominal = NOMINAL["hbm_gbs"]
     return {"kernel": name, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
             "frac": achieved / peak, "traffic": traffic, "peak_source": peaks["source"],
+            "frac_of_nominal": achieved / nominal, "nominal_peak": nominal,
             "share": e["ms"] / sum(v["ms"] for v in table.values())}
 
 
@@ -476,6 +485,7 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
     value = world * fl["tower"] / (ms * 1e-3) / 1e12
     block_tflops = fl["block"] / (block_ms * 1e-3) / 1e12
     ideal_block_ms = (fl["block_gemm"] / (2 * peaks["bf16"]) + fl["block_attn"] / peaks["bf16"]) / 1e9
+    ideal_nominal_ms = (fl["block_gemm"] / NOMINAL["fp8"] + fl["block_attn"] / NOMINAL["bf16"]) / 1e9
     h2d = x_host.numel() * x_host.element_size()
     d2h = sum(t.numel() * t.element_size() for t in taps)
     line = {
@@ -489,6 +499,8 @@ def run_gpu(args, rank: int, world: int, local_rank: int):
         "block_ms": block_ms, "block_tflops": block_tflops,
         "block_frac_of_peak": ideal_block_ms / block_ms,
         "block_ideal_ms": ideal_block_ms,
+        "block_frac_of_nominal_peak": ideal_nominal_ms / block_ms,
+        "block_ideal_nominal_ms": ideal_nominal_ms,
         "tower_ms": ms,
         "block_bf16_ms": block_bf16_ms,
         "mixed_tower_ms": mixed_ms,

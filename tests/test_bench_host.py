@@ -44,3 +44,41 @@ def test_clock_summary():
     s.lines = ["1200, 1965, 700, Active, Not Active, Active, Not Active"]
     assert s.summary()["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
     assert bench.ClockSampler(0).summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+def _table():
+    # per-kernel event sums as bench.py collects them (two timed steps' worth)
+    return {"attention": {"launches": 54, "ms": 15.34, "flops": 54 * 180.35e9, "bytes": 54 * 57.7e6},
+            "fp8_block_gemm": {"launches": 232, "ms": 10.48, "flops": 232 * 50e9, "bytes": 232 * 50e6},
+            "ln_quant": {"launches": 116, "ms": 3.31, "flops": 0.0, "bytes": 116 * 21.9e6}}
+
+
+def test_roofline_of_the_dominant_kernel():
+    peaks = {"hbm_gbs": 6455.6, "bf16": 1649.5, "bf16_sustained": 1415.6, "source": "measured"}
+    r = bench.roofline(_table(), peaks)
+    per_launch_s = 15.34e-3 / 54
+    assert r["kernel"] == "attention" and r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["achieved"] - 180.35e9 / per_launch_s / 1e12) < 1e-9
+    assert r["peak"] == 1415.6 and abs(r["frac"] - r["achieved"] / 1415.6) < 1e-12
+    assert r["nominal_peak"] == 2250.0 and abs(r["frac_of_nominal"] - r["achieved"] / 2250.0) < 1e-12
+    assert abs(r["share"] - 15.34 / (15.34 + 10.48 + 3.31)) < 1e-12
+    # a GEMM-dominated table takes the FP8 peak (measured bf16 x 2), an HBM-bound one GB/s
+    t = _table()
+    t["fp8_block_gemm"]["ms"] = 40.0
+    g = bench.roofline(t, peaks)
+    assert g["kernel"] == "fp8_block_gemm" and g["peak"] == 2 * 1415.6 and g["nominal_peak"] == 4500.0
+    t["ln_quant"]["ms"] = 100.0
+    h = bench.roofline(t, peaks)
+    assert h["bound"] == "hbm" and h["unit"] == "GB/s" and h["peak"] == 6455.6
+    assert abs(h["achieved"] - 21.9e6 / (100e-3 / 116) / 1e9) < 1e-9
+
+
+def test_roofline_traffic_only_for_the_profiled_source(monkeypatch):
+    """ncu traffic is reported only while the kernel source still hashes to the one profiled."""
+    import json
+    peaks = bench.load_peaks()
+    rec = json.load(open(os.path.join(ROOT, "profiles", "traffic.json")))["attention"]
+    monkeypatch.setattr(bench, "_source_sha", lambda rel: rec["source_sha"])
+    assert bench.roofline(_table(), peaks)["traffic"] == rec["bytes_per_launch"]
+    monkeypatch.setattr(bench, "_source_sha", lambda rel: "0" * 16)
+    assert bench.roofline(_table(), peaks)["traffic"] is None
