@@ -129,7 +129,8 @@ typedef struct {
  * Outputs q [M, K] and s[kb * lds + m].  K % 16 == 0, lds >= M. */
 int vit_quant_act(const void* x, int M, int K, int ldx, uint8_t* q, float* s, int lds, void* stream);
 
-/* 128x128-block FP8 weight quantisation (same convention, one scale per block).
+/* 128x128-block FP8 weight quantisation ([FRT] introduction: block-128 W8A8
+ * linears; scale convention [TRT]) (same convention, one scale per block).
  * w: bf16 [N, K] -> q [N, K], s [ceil(N/128), ceil(K/128)].  Set-up step. */
 int vit_quant_weight(const void* w, int N, int K, uint8_t* q, float* s, void* stream);
 
@@ -179,7 +180,8 @@ int vit_rope_table(const int32_t* pos_hw, int n_tokens, float theta, float* cos_
  * of 8) at the same tensor-core rate. */
 #define VITQ_V_FP16 1
 
-/* Apply the rotary in place to the q and k parts of qkv bf16 [n, 3, 16, 72]:
+/* 2D rotary ([FRT] s3, applied after the QKV projection; [VE] head_dim 72).
+ * Apply the rotary in place to the q and k parts of qkv bf16 [n, 3, 16, 72]:
  * pairs (j, j+36): x'_j = x_j cos - x_(j+36) sin, x'_(j+36) = x_(j+36) cos + x_j sin,
  * fp32 arithmetic, one rounding to bf16.  flags = VITQ_V_FP16 also converts the
  * v part to fp16 in place; flags = 0 leaves it untouched. */
@@ -277,16 +279,19 @@ int vit_tower_forward(const vitq_tower_weights* w, void* x, const int32_t* grid_
                       void* const* taps, void* ws, size_t ws_bytes, void* stream);
 size_t vitq_tower_workspace_bytes(int n_tokens_max, int n_images_max);
 
-/* bf16 block, in place on x bf16 [n_tokens, 1152]: LN1 (bf16) -> QKV bf16 GEMM +
- * bias -> RoPE -> attention -> proj bf16 GEMM + bias + x -> LN2 (bf16) -> fc1
- * bf16 GEMM + bias -> GELU (bf16) -> fc2 bf16 GEMM + bias + residual.  Arguments
- * as vit_block_forward; ws >= vitq_block_workspace_bytes(n_tokens). */
+/* bf16 block ([FRT] s4: the first three blocks keep bf16 weights and
+ * activations; the per-block chain of [FRT] s3), in place on x bf16
+ * [n_tokens, 1152]: LN1 (bf16) -> QKV bf16 GEMM + bias -> RoPE -> attention ->
+ * proj bf16 GEMM + bias + x -> LN2 (bf16) -> fc1 bf16 GEMM + bias -> GELU (bf16)
+ * -> fc2 bf16 GEMM + bias + residual.  Arguments as vit_block_forward;
+ * ws >= vitq_block_workspace_bytes(n_tokens). */
 int vit_block_forward_bf16(const vitq_block_weights_bf16* w, void* x, int n_tokens, const int32_t* cu_seqlens,
                            int n_seqs, int max_seqlen, const float* cos_sin, void* ws, size_t ws_bytes,
                            void* stream);
 
-/* bf16 2x2 merger: as vit_merger_forward with bf16 LayerNorm output, bf16 fc1
- * and fc2 and a bf16 GELU.  ws >= vitq_merger_bf16_workspace_bytes(n_tokens). */
+/* bf16 2x2 merger ([FRT] s4: the mergers keep bf16): as vit_merger_forward
+ * with bf16 LayerNorm output, bf16 fc1 and fc2 and a bf16 GELU.
+ * ws >= vitq_merger_bf16_workspace_bytes(n_tokens). */
 int vit_merger_forward_bf16(const vitq_merger_weights_bf16* w, const void* x, int n_tokens, void* out, void* ws,
                             size_t ws_bytes, void* stream);
 size_t vitq_merger_bf16_workspace_bytes(int n_tokens);
