@@ -26,17 +26,20 @@ _vp, _i, _f, _sz = C.c_void_p, C.c_int, C.c_float, C.c_size_t
 
 
 class BlockWeights(C.Structure):
+    """vitq_block_weights: device pointers of one FP8 block."""
     _fields_ = [(n, _vp) for n in (
         "norm1_w", "norm1_b", "qkv_q", "qkv_s", "qkv_b", "proj_q", "proj_s", "proj_b",
         "norm2_w", "norm2_b", "fc1_q", "fc1_s", "fc1_b", "fc2_q", "fc2_s", "fc2_b")]
 
 
 class MergerWeights(C.Structure):
+    """vitq_merger_weights: device pointers of one FP8 merger."""
     _fields_ = [(n, _vp) for n in (
         "norm_w", "norm_b", "fc1_q", "fc1_s", "fc1_b", "fc2_q", "fc2_s", "fc2_b")]
 
 
 class TowerWeights(C.Structure):
+    """vitq_tower_weights: 27 blocks and 4 mergers."""
     _fields_ = [("blocks", BlockWeights * N_BLOCKS), ("mergers", MergerWeights * 4)]
 
 
@@ -44,16 +47,19 @@ BF16_HEAD_BLOCKS = 3
 
 
 class BlockWeightsBf16(C.Structure):
+    """vitq_block_weights_bf16: device pointers of one bf16 block."""
     _fields_ = [(n, _vp) for n in (
         "norm1_w", "norm1_b", "qkv_w", "qkv_b", "proj_w", "proj_b",
         "norm2_w", "norm2_b", "fc1_w", "fc1_b", "fc2_w", "fc2_b")]
 
 
 class MergerWeightsBf16(C.Structure):
+    """vitq_merger_weights_bf16: device pointers of one bf16 merger."""
     _fields_ = [(n, _vp) for n in ("norm_w", "norm_b", "fc1_w", "fc1_b", "fc2_w", "fc2_b")]
 
 
 class TowerWeightsMixed(C.Structure):
+    """vitq_tower_weights_mixed: bf16 blocks 1-3 and mergers, FP8 blocks 4-27."""
     _fields_ = [("head", BlockWeightsBf16 * BF16_HEAD_BLOCKS),
                 ("blocks", BlockWeights * (N_BLOCKS - BF16_HEAD_BLOCKS)),
                 ("mergers", MergerWeightsBf16 * 4)]
@@ -116,6 +122,7 @@ def load(path: str = LIB_PATH):
 
 
 class VitqError(RuntimeError):
+    """A non-zero vitq_status, or a tensor argument the C side cannot take."""
     pass
 
 
@@ -175,14 +182,18 @@ def _stream(stream=None):
 
 
 def launch_count() -> int:
+    """Kernel launches issued by the library since it was loaded."""
     return int(load().vitq_launch_count())
 
 
 def device_error(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device error word: 0, 7 after a
+    bounded wait timed out, 5 if synchronising failed."""
     return int(load().vitq_get_device_error(_stream(stream)))
 
 
 def profile_start():
+    """Start bracketing every library launch with CUDA events (not during stream capture)."""
     load().vitq_profile_start()
 
 
@@ -201,6 +212,7 @@ def profile_stop() -> list:
 
 
 def selftest_wait_timeout(limit_us: int = 20000, stream=None):
+    """Launch a kernel whose pipeline wait can never complete; it gives up after limit_us."""
     _check(load().vitq_selftest_wait_timeout(limit_us, _stream(stream)), "vitq_selftest_wait_timeout")
 
 
@@ -230,6 +242,7 @@ def quant_weight(w: torch.Tensor, stream=None):
 
 
 def ln_quant(x, gamma, beta, eps: float = 1e-6, stream=None):
+    """LayerNorm of bf16 x [M, K] (rows dense), rounded to bf16 and 1x128 FP8-quantised -> (codes, scales)."""
     M, K = _arg(x, "x", _bf16, (None, None), rows=True).shape
     _arg(gamma, "gamma", _bf16, (K,))
     _arg(beta, "beta", _bf16, (K,))
@@ -241,6 +254,7 @@ def ln_quant(x, gamma, beta, eps: float = 1e-6, stream=None):
 
 
 def gelu_quant(f, stream=None):
+    """GELU(tanh) of bf16 f [M, K] (rows dense), rounded to bf16 and 1x128 FP8-quantised -> (codes, scales)."""
     M, K = _arg(f, "f", _bf16, (None, None), rows=True).shape
     q = torch.empty((M, K), dtype=torch.uint8, device=f.device)
     s, lds = _scales((K + 127) // 128, M, f.device)
@@ -286,6 +300,7 @@ def bf16_gemm(a, w, bias=None, residual=None, out=None, stream=None):
 
 
 def rope_table(pos_hw: torch.Tensor, theta: float = 10000.0, stream=None):
+    """cos / sin table fp32 [n, 72] for int32 (row, col) positions [n, 2]."""
     n = _arg(pos_hw, "pos_hw", _i32, (None, 2)).shape[0]
     cs = torch.empty((n, 72), dtype=torch.float32, device=pos_hw.device)
     _check(load().vit_rope_table(_p(pos_hw), n, theta, _p(cs), _stream(stream)), "vit_rope_table")
@@ -315,6 +330,7 @@ def positions(grids, device="cuda", stream=None):
 
 def attention_varlen(qkv, cu_seqlens, max_seqlen: int, scale: float | None = None, out=None, flags: int = 0,
                      stream=None):
+    """Block-diagonal attention over bf16 qkv [n, 3456] with int32 cu_seqlens -> bf16 [n, 1152]."""
     n = _arg(qkv, "qkv", _bf16, (None, QKV)).shape[0]
     _cu(cu_seqlens)
     if out is None:
@@ -375,6 +391,8 @@ class DeviceBlock:
 
 
 class DeviceMerger:
+    """Device-resident merger weights (bf16 vectors, FP8 codes, fp32 scales) and their C struct."""
+
     def __init__(self, params: dict, device="cuda", stream=None):
         t = _weights(params, MERGER_SHAPES, device)
         self.t = t
@@ -392,6 +410,8 @@ class DeviceBlockBf16:
 
 
 class DeviceMergerBf16:
+    """Device-resident bf16 merger weights and their C struct."""
+
     def __init__(self, params: dict, device="cuda"):
         self.t = _weights(params, MERGER_SHAPES, device)
         self.struct = MergerWeightsBf16(**{f: self.t[f].data_ptr() for f, _ in MergerWeightsBf16._fields_})
@@ -423,10 +443,12 @@ def block_forward_bf16_(blk: DeviceBlockBf16, x, cu_seqlens, max_seqlen, cos_sin
 
 
 def merger_bf16_workspace_bytes(n: int) -> int:
+    """Workspace bytes of vit_merger_forward_bf16 at n input tokens (0 if n is out of range)."""
     return int(load().vitq_merger_bf16_workspace_bytes(n))
 
 
 def merger_forward_bf16(mg: DeviceMergerBf16, x, ws, out=None, stream=None):
+    """bf16 2x2 merger of bf16 x [n, 1152] -> [n/4, 2048]."""
     n = _x(x)
     _ws(ws)
     if out is None:
@@ -470,18 +492,22 @@ def patch_embed(pixels, grids, w, b, pos_table, out=None, ws=None, stream=None):
 
 
 def block_workspace_bytes(n: int) -> int:
+    """Workspace bytes of vit_block_forward at n tokens (0 if n is out of range)."""
     return int(load().vitq_block_workspace_bytes(n))
 
 
 def merger_workspace_bytes(n: int) -> int:
+    """Workspace bytes of vit_merger_forward at n input tokens (0 if n is out of range)."""
     return int(load().vitq_merger_workspace_bytes(n))
 
 
 def tower_workspace_bytes(n: int, n_images: int) -> int:
+    """Workspace bytes of the tower at up to n tokens in up to n_images images (0 if out of range)."""
     return int(load().vitq_tower_workspace_bytes(n, n_images))
 
 
 def workspace(nbytes: int, device="cuda"):
+    """A uint8 device buffer of nbytes (at least 1) to pass as a workspace."""
     return torch.empty((max(nbytes, 1),), dtype=torch.uint8, device=device)
 
 
@@ -497,6 +523,7 @@ def block_forward_(blk: DeviceBlock, x, cu_seqlens, max_seqlen, cos_sin, ws, str
 
 
 def merger_forward(mg: DeviceMerger, x, ws, out=None, stream=None):
+    """FP8 2x2 merger of bf16 x [n, 1152] -> [n/4, 2048]."""
     n = _x(x)
     _ws(ws)
     if out is None:
@@ -520,6 +547,8 @@ def merger_forward_static(mg: DeviceMerger, x, out):
 
 
 class DeviceTower:
+    """27 DeviceBlock and 4 DeviceMerger objects and the vitq_tower_weights struct over them."""
+
     def __init__(self, blocks, mergers):
         self.blocks, self.mergers = blocks, mergers
         self.struct = TowerWeights()
