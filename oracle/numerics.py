@@ -23,7 +23,8 @@ E4M3_NAN = 0x7F
 
 
 def bf16_round(x) -> np.ndarray:
-    """Round fp64 values to the nearest bf16 value (ties to even), returned as fp64."""
+    """Round fp64 values to the nearest bf16 value (ties to even), returned as fp64
+    (bfloat16 format definition; the block's activations are bf16 [FRT s3])."""
     x = np.asarray(x, dtype=np.float64)
     m, e = np.frexp(x)                       # x = m * 2**e, 0.5 <= |m| < 1
     out = np.ldexp(np.rint(m * 256.0), e - 8)  # 8 significant bits
@@ -52,12 +53,14 @@ _E4M3_TABLE = _e4m3_value(np.arange(256))
 
 
 def e4m3_decode(codes) -> np.ndarray:
-    """Exact value of each E4M3 code (uint8 array) as fp64; 0x7F/0xFF give NaN."""
+    """Exact value of each E4M3 code (uint8 array) as fp64; 0x7F/0xFF give NaN
+    (OCP E4M3 definition; FP8 E4M3 GEMM operands [FRT s1])."""
     return _E4M3_TABLE[np.asarray(codes).astype(np.uint8)]
 
 
 def e4m3_encode(v) -> np.ndarray:
-    """E4M3 code of each fp32 value: round to nearest even, saturate to +-448."""
+    """E4M3 code of each fp32 value: round to nearest even, saturate to +-448
+    (OCP E4M3 definition; the 448 of the scale amax / 448 [TRT recipe])."""
     v = np.asarray(v, dtype=np.float32)
     sign = np.signbit(v).astype(np.int64) << 7
     a = np.abs(v.astype(np.float64))

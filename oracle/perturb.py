@@ -9,7 +9,9 @@ near 1e-2, and over the 27-block tower to several 1e-2 whatever the size of the
 original difference.  A CUDA implementation cannot reproduce the oracle's
 fp64 rounding of every intermediate, so block-, merger- and tower-level outputs
 are compared against the drift the oracle itself shows when one of its
-intermediate roundings is moved by a tiny amount.
+intermediate roundings is moved by a tiny amount.  (The pages show the same growth with
+depth: FP8 against bf16 image-embedding cosines fall from block 8 to the last DeepStack
+tap [FRT s4].)
 
 Three perturbations are modelled, each a documented change of a rounding point:
   gemm_fp32_promotion : the per-128-K partial sums (exact) are scaled and summed
@@ -30,7 +32,8 @@ from .numerics import bf16_round, e4m3_decode
 
 
 def fp8_block_gemm_fp32_promotion(qa, sa, qw, sw, bias=None, residual=None):
-    """fp8_block_gemm with the K-block scaling and the outer sum in fp32."""
+    """fp8_block_gemm with the K-block scaling and the outer sum in fp32 (the fp32
+    accumulation of the FP8 GEMMs [FRT s1, s3])."""
     a = e4m3_decode(qa)
     w = e4m3_decode(qw)
     M, K = qa.shape
@@ -49,7 +52,8 @@ def fp8_block_gemm_fp32_promotion(qa, sa, qw, sw, bias=None, residual=None):
 
 
 def attention_bf16_p(qkv, cu_seqlens, heads: int = 16, head_dim: int = 72, scale=None):
-    """attention_varlen with P rounded to bf16 before the P.V product and the row sum."""
+    """attention_varlen with P rounded to bf16 before the P.V product and the row sum (a bf16
+    flash-attention kernel [FRT s3])."""
     qkv = np.asarray(qkv, np.float64)
     n = qkv.shape[0]
     scale = 1.0 / math.sqrt(head_dim) if scale is None else scale
@@ -65,7 +69,8 @@ def attention_bf16_p(qkv, cu_seqlens, heads: int = 16, head_dim: int = 72, scale
 
 
 def bf16_gemm_fp32(a, w, bias=None, residual=None):
-    """bf16_gemm with the product summed, and bias and residual added, in fp32."""
+    """bf16_gemm with the product summed, and bias and residual added, in fp32 (the bf16
+    linears of the first blocks and the mergers [FRT s4])."""
     acc = np.asarray(a, np.float32) @ np.asarray(w, np.float32).T
     if bias is not None:
         acc = acc + np.asarray(bias, np.float32)[None, :]

@@ -52,7 +52,8 @@ QBLK = 128                       # FP8 scaling block (1x128 activations, 128x128
 # --------------------------------------------------------------------------
 
 def quant_act(y) -> tuple:
-    """Per-row, per-128-column FP8 quantisation of bf16-valued activations.
+    """Per-row, per-128-column FP8 quantisation of bf16-valued activations
+    [FRT s3: per-token / per-128-K-block activation quant; TRT recipe: scale amax / 448].
 
     Returns (codes uint8 [M, K], scales float32 [ceil(K/128), M]).
     """
@@ -75,7 +76,8 @@ def quant_act(y) -> tuple:
 
 
 def quant_weight(w) -> tuple:
-    """Per-128x128-block FP8 quantisation of a bf16-valued weight [N, K].
+    """Per-128x128-block FP8 quantisation of a bf16-valued weight [N, K]
+    [FRT introduction: block-128 W8A8 linears; TRT recipe: scale amax / 448].
 
     Returns (codes uint8 [N, K], scales float32 [ceil(N/128), ceil(K/128)]).
     """
@@ -99,7 +101,7 @@ def quant_weight(w) -> tuple:
 
 
 def dequant_act(codes, scales) -> np.ndarray:
-    """Value represented by activation codes and their 1x128 scales (fp64)."""
+    """Value represented by activation codes and their 1x128 scales (fp64) [FRT s3]."""
     M, K = codes.shape
     col_scale = np.repeat(scales.astype(np.float64), QBLK, axis=0)[:K].T   # [M, K]
     return e4m3_decode(codes) * col_scale
@@ -115,7 +117,8 @@ def fp8_block_gemm(qa, sa, qw, sw, bias=None, residual=None) -> np.ndarray:
     P_kb is the sum over the 128 columns of K block kb of decoded code
     products.  Each product is a multiple of 2**-18 below 2**18, so every
     partial sum of 128 of them is exact in fp64 whatever the order; the
-    outer sum over K blocks is taken in fp64.
+    outer sum over K blocks is taken in fp64.  [FRT s1, s3: FP8 block-128 W8A8
+    GEMMs with the bias (and residual) added in the same kernel; VE vision_gemm_bias.]
     """
     M, K = qa.shape
     N = qw.shape[0]
@@ -156,7 +159,7 @@ def bf16_gemm(a, w, bias=None, residual=None) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 def layernorm_f64(x, gamma, beta, eps: float = 1e-6) -> np.ndarray:
-    """Biased-variance LayerNorm in fp64, not rounded."""
+    """Biased-variance LayerNorm in fp64, not rounded [FRT s3 block chain; VE norm1_w / norm1_b]."""
     x = np.asarray(x, np.float64)
     mu = x.mean(axis=1, keepdims=True)
     var = ((x - mu) ** 2).mean(axis=1, keepdims=True)
@@ -164,11 +167,13 @@ def layernorm_f64(x, gamma, beta, eps: float = 1e-6) -> np.ndarray:
 
 
 def layernorm(x, gamma, beta, eps: float = 1e-6) -> np.ndarray:
+    """LayerNorm rounded once to bf16, the block's normalised activation [FRT s3]."""
     return bf16_round(layernorm_f64(x, gamma, beta, eps))
 
 
 def gelu_tanh_f64(x) -> np.ndarray:
-    """GELU(tanh) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3), in fp64, not rounded.
+    """GELU(tanh) = 0.5 x (1 + tanh(u)), u = sqrt(2/pi) (x + 0.044715 x^3), in fp64, not rounded
+    [FRT s3: GELU(tanh)].
 
     Evaluated as x / (1 + exp(-2u)), which equals 0.5 x (1 + tanh(u)) exactly
     (1 + tanh(u) = 2 / (1 + exp(-2u))) but does not cancel for u << 0, where
@@ -181,6 +186,7 @@ def gelu_tanh_f64(x) -> np.ndarray:
 
 
 def gelu_tanh(x) -> np.ndarray:
+    """GELU(tanh) rounded once to bf16 [FRT s3]."""
     return bf16_round(gelu_tanh_f64(x))
 
 
@@ -199,7 +205,8 @@ def gelu_quant(f) -> tuple:
 # --------------------------------------------------------------------------
 
 def patch_positions(h: int, w: int) -> np.ndarray:
-    """(row, col) of each patch of an h x w grid in token order, int64 [h*w, 2].
+    """(row, col) of each patch of an h x w grid in token order, int64 [h*w, 2]
+    [FRT s3: 2D positions for the rotary and the 2x2 merger; VE MergerLayer].
 
     Even grids use 2x2-block order: block (br, bc) in row-major order, and
     inside it (0,0), (0,1), (1,0), (1,1).  Odd grids use row-major order.
@@ -219,7 +226,7 @@ def patch_positions(h: int, w: int) -> np.ndarray:
 
 
 def packed_positions(grids) -> tuple:
-    """Positions of all packed images and their cu_seqlens."""
+    """Positions of all packed images and their cu_seqlens [FRT s5: one attention window per image]."""
     pos = [patch_positions(h, w) for h, w in grids]
     cu = [0]
     for h, w in grids:
@@ -237,7 +244,8 @@ POS_GRID = 48
 
 
 def pos_embed_interp(table, h: int, w: int) -> np.ndarray:
-    """Bilinear interpolation of the learned 48 x 48 position table to an h x w patch grid.
+    """Bilinear interpolation of the learned 48 x 48 position table to an h x w patch grid
+    [FRT s3: interpolated pos_embed; VE num_grid_per_side 48].
 
     Sample points run from corner to corner: grid row r of h sits at table row
     r * 47 / (h - 1) (0 when h = 1), likewise for columns; each value mixes the
@@ -262,6 +270,7 @@ def patch_embed(pixels, w, b, table, grids) -> np.ndarray:
     the interpolated position embedding of each patch rounded to bf16.
 
     pixels: [n, 1536] patch rows (already normalised and patchified); w [1152, 1536].
+    [FRT s3: patch_embed then the interpolated pos_embed; VE PATCH_DIM 1536.]
     """
     pos = []
     for h, wd in grids:
@@ -272,7 +281,7 @@ def patch_embed(pixels, w, b, table, grids) -> np.ndarray:
 
 
 def rope_inv_freq(head_dim: int = 72, theta: float = 10000.0) -> np.ndarray:
-    """head_dim/4 frequencies theta**(-2i/(head_dim/2)), fp64."""
+    """head_dim/4 frequencies theta**(-2i/(head_dim/2)), fp64 [VE rope_inv_freq; FRT s3 2D RoPE]."""
     half = head_dim // 2
     i = np.arange(half // 2, dtype=np.float64)
     return theta ** (-2.0 * i / half)
@@ -280,14 +289,15 @@ def rope_inv_freq(head_dim: int = 72, theta: float = 10000.0) -> np.ndarray:
 
 def rope_angles(pos, head_dim: int = 72, theta: float = 10000.0) -> np.ndarray:
     """Rotation angle of pair j (0 <= j < head_dim/2): row*f_j for the first
-    head_dim/4 pairs, col*f_(j - head_dim/4) for the rest.  fp64 [n, head_dim/2]."""
+    head_dim/4 pairs, col*f_(j - head_dim/4) for the rest.  fp64 [n, head_dim/2].
+    [FRT s3: 2D RoPE; VE rope_inv_freq.]"""
     f = rope_inv_freq(head_dim, theta)
     pos = np.asarray(pos, np.float64)
     return np.concatenate([pos[:, :1] * f[None, :], pos[:, 1:2] * f[None, :]], axis=1)
 
 
 def rope_rotate(x, angles) -> np.ndarray:
-    """rotate_half rotary on the last axis of x [n, ..., d]; pairs (j, j + d/2).
+    """rotate_half rotary on the last axis of x [n, ..., d]; pairs (j, j + d/2) [FRT s3].
 
     x'_j = x_j cos a_j - x_(j+d/2) sin a_j,  x'_(j+d/2) = x_(j+d/2) cos a_j + x_j sin a_j.
     fp64, not rounded.  angles is [n, d/2] and broadcasts over middle axes.
@@ -304,7 +314,8 @@ def rope_rotate(x, angles) -> np.ndarray:
 
 def apply_rope_qkv(qkv, pos, heads: int = 16, head_dim: int = 72, theta: float = 10000.0) -> np.ndarray:
     """Rotate the q and k parts of a packed qkv [n, 3*heads*head_dim] ([n, 3, heads, head_dim]
-    order); v is unchanged.  Result rounded to bf16."""
+    order); v is unchanged.  Result rounded to bf16.  [FRT s3: RoPE on q and k after
+    the QKV projection.]"""
     qkv = np.asarray(qkv, np.float64)
     n = qkv.shape[0]
     t = qkv.reshape(n, 3, heads, head_dim)
@@ -320,7 +331,8 @@ def apply_rope_qkv(qkv, pos, heads: int = 16, head_dim: int = 72, theta: float =
 # --------------------------------------------------------------------------
 
 def attention_varlen(qkv, cu_seqlens, heads: int = 16, head_dim: int = 72, scale=None) -> np.ndarray:
-    """softmax(q k^T * scale) v per segment and head, fp64; output [n, heads*head_dim] rounded to bf16."""
+    """softmax(q k^T * scale) v per segment and head, fp64; output [n, heads*head_dim] rounded to bf16
+    [FRT s3: full bidirectional attention; s5: cu_seqlens segments]."""
     qkv = np.asarray(qkv, np.float64)
     n = qkv.shape[0]
     if scale is None:
@@ -346,7 +358,8 @@ def attention_varlen(qkv, cu_seqlens, heads: int = 16, head_dim: int = 72, scale
 # --------------------------------------------------------------------------
 
 def quantize_block_weights(p: dict) -> dict:
-    """FP8 codes + 128x128 scales of the four linear layers of a block (bf16-valued inputs)."""
+    """FP8 codes + 128x128 scales of the four linear layers of a block (bf16-valued inputs)
+    [FRT introduction: block-128 W8A8]."""
     q = dict(p)
     for name in ("qkv", "proj", "fc1", "fc2"):
         q[name + "_q"], q[name + "_s"] = quant_weight(p[name + "_w"])
@@ -354,6 +367,7 @@ def quantize_block_weights(p: dict) -> dict:
 
 
 def quantize_merger_weights(p: dict) -> dict:
+    """FP8 codes + 128x128 scales of the merger's fc1 and fc2 [FRT introduction, s3 merger]."""
     q = dict(p)
     for name in ("fc1", "fc2"):
         q[name + "_q"], q[name + "_s"] = quant_weight(p[name + "_w"])
@@ -365,6 +379,8 @@ def block_forward(x, w: dict, cu_seqlens, pos, eps: float = 1e-6, keep: bool = F
     the FP8 codes/scales of the linears (see quantize_block_weights).
 
     Returns x2, or (x2, dict of every intermediate) with keep=True.
+    [FRT s3: the per-block chain LN -> QKV -> RoPE -> attention -> proj + residual ->
+    LN -> fc1 -> GELU -> fc2 + residual; VE ViTBlock.]
     """
     x = np.asarray(x, np.float64)
     st = {}
@@ -413,7 +429,8 @@ def merger_forward_bf16(x, w: dict, eps: float = 1e-6, keep: bool = False):
 
 
 def merger_forward(x, w: dict, eps: float = 1e-6, keep: bool = False):
-    """2x2 merger: 4 consecutive rows -> one 4608 row, LayerNorm, fc1, GELU, fc2."""
+    """2x2 merger: 4 consecutive rows -> one 4608 row, LayerNorm, fc1, GELU, fc2
+    [FRT s3: 2x2 merger on the DeepStack taps; VE MergerLayer]."""
     x = np.asarray(x, np.float64)
     n, c = x.shape
     xm = x.reshape(n // 4, 4 * c)
@@ -432,6 +449,8 @@ def tower_forward(x, blocks, mergers, grids, taps_after=(8, 16, 24, 27), eps: fl
     blocks: list of block weight dicts, each either quantised (quantize_block_weights: FP8
     block) or the bf16 weights themselves (no "qkv_q": bf16 block); mergers likewise.
     Returns the list of merger outputs (one per tap).
+    [FRT s3: DeepStack taps after blocks 8, 16, 24 and the final merger; VE VisionEncoder
+    deepstack indexes.]
     """
     pos, cu = packed_positions(grids)
     h = np.asarray(x, np.float64)
