@@ -253,6 +253,10 @@ bool merger_weights_ok(const vitq_merger_weights* w) {
 // Algorithmic HBM bytes of the row kernels (read bf16 rows, write codes + scales).
 inline double quant_bytes(double M, double K) { return M * K * 2 + M * K + M * ((K + 127) / 128) * 4; }
 
+// One FP8 block in place on x ("Qwen3-VL-8B on RTX 5090", section 3, the per-block
+// chain; "spark_model/layers/vision_encoder.rs", ViTBlock): LN1+quant, QKV GEMM + bias,
+// rotary (v to fp16), attention, quant, proj GEMM + bias + x, LN2+quant, fc1 GEMM +
+// bias, GELU+quant, fc2 GEMM + bias + x1.
 int block_impl(const vitq_block_weights* w, __nv_bfloat16* x, int n, const int32_t* cu, int n_seqs,
                int max_seqlen, const float* cs, const BlockWs& b, int num_sms, double attn_sumsq,
                cudaStream_t st) {
@@ -285,6 +289,9 @@ int block_impl(const vitq_block_weights* w, __nv_bfloat16* x, int n, const int32
                       num_sms, st);
 }
 
+// One FP8 2x2 merger ("Qwen3-VL-8B on RTX 5090", section 3; vision_encoder.rs,
+// MergerLayer): four consecutive rows read as one 4608 row, LN+quant, fc1 + bias,
+// GELU+quant, fc2 + bias.
 int merger_impl(const vitq_merger_weights* w, const __nv_bfloat16* x, int n, __nv_bfloat16* out,
                 const MergerWs& m, int num_sms, cudaStream_t st) {
   using bf = __nv_bfloat16;
@@ -319,7 +326,8 @@ bool merger_bf16_weights_ok(const vitq_merger_weights_bf16* w) {
   return true;
 }
 
-// bf16 block: the LayerNorm outputs go to the codes region of the block
+// bf16 block ("Qwen3-VL-8B on RTX 5090", section 4: the first three blocks keep
+// bf16): the LayerNorm outputs go to the codes region of the block
 // workspace (n * 4304 bytes >= n * 1152 bf16), GELU runs in place on the fc1 output.
 int block_bf16_impl(const vitq_block_weights_bf16* w, __nv_bfloat16* x, int n, const int32_t* cu, int n_seqs,
                     int max_seqlen, const float* cs, const BlockWs& b, int num_sms, double attn_sumsq,
@@ -352,6 +360,7 @@ int block_bf16_impl(const vitq_block_weights_bf16* w, __nv_bfloat16* x, int n, c
                            num_sms, st);
 }
 
+// bf16 2x2 merger ("Qwen3-VL-8B on RTX 5090", section 4: the mergers keep bf16).
 int merger_bf16_impl(const vitq_merger_weights_bf16* w, const __nv_bfloat16* x, int n, __nv_bfloat16* out,
                      const MergerBf16Ws& m, int num_sms, cudaStream_t st) {
   using bf = __nv_bfloat16;
@@ -628,7 +637,8 @@ int vit_merger_forward(const vitq_merger_weights* w, const void* x, int n_tokens
 namespace vitq {
 namespace {
 
-// Tower driver: positions and rope table, then the 27 blocks with the 4 mergers
+// Tower driver ("Qwen3-VL-8B on RTX 5090", section 3, DeepStack taps; vision_encoder.rs,
+// VisionEncoder): positions and rope table, then the 27 blocks with the 4 mergers
 // after blocks 8, 16, 24 and 27.  run_block(blk, ...) and run_merger(tap, ...)
 // pick each block's and merger's precision.
 template <class BlockFn, class MergerFn>

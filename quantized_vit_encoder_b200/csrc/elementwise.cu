@@ -170,6 +170,8 @@ __global__ void __launch_bounds__(128, 12) quant_act_kernel(const __nv_bfloat16*
 }
 
 // --------------------------------------------------------- LayerNorm + quant
+// "Qwen3-VL-8B on RTX 5090", section 3: LayerNorm with the FP8 quantisation of
+// its bf16 output fused in (the normalised activation never goes to HBM).
 // A half warp per row (lane l of the half holds columns 128c + 8l, so each
 // 128-column group is one chunk c across the half warp), eight rows per CTA;
 // gamma, beta and the bracket term below are staged once per CTA in shared
@@ -311,6 +313,8 @@ __global__ void __launch_bounds__(16 * kLnRows, 6)
 }
 
 // ------------------------------------------------------------- GELU + quant
+// "Qwen3-VL-8B on RTX 5090", section 3: GELU(tanh) on the fc1 output with the FP8
+// quantisation for fc2 fused in.
 // GELU(tanh) = 0.5 x (1 + tanh(u)) = x / (1 + exp(-2u)), u = sqrt(2/pi)(x + 0.044715 x^3).
 // Its input is a bf16 value (the rounded fc1 output), so the bf16 result is a
 // function of 16 bits: g_gelu_table holds it for every bf16 bit pattern,
@@ -434,6 +438,9 @@ __global__ void quant_weight_kernel(const __nv_bfloat16* __restrict__ w, int N, 
 }
 
 // --------------------------------------------------------------- 2D rotary
+// "Qwen3-VL-8B on RTX 5090", section 3 (2D rotate_half rotary after the QKV
+// projection) and "spark_model/layers/vision_encoder.rs" (rope_inv_freq: head_dim/4
+// = 18 frequencies, used for the row and for the column).
 // Table layout: cos_sin[t * 72 + j] = cos(angle_j), cos_sin[t * 72 + 36 + j] = sin(angle_j),
 // angle_j = row * f_j (j < 18), col * f_(j-18) (18 <= j < 36), f_i = theta^(-2i/36).
 
@@ -564,6 +571,10 @@ __global__ void __launch_bounds__(144) pos_interp_kernel(GridList grids, const _
   *reinterpret_cast<uint4*>(out + (size_t)t * 1152 + d0) = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
+// (row, col) of every patch of the packed images and the segment offsets
+// ("Qwen3-VL-8B on RTX 5090", section 5: each image is its own attention window).
+// Even grids are walked in 2x2-block order, so the merger's four neighbours are
+// consecutive rows; odd grids row-major.
 __global__ void positions_kernel(GridList grids, int n_total, int32_t* __restrict__ pos,
                                  int32_t* __restrict__ cu) {
   pdl_trigger();
