@@ -24,6 +24,14 @@
  *  - Arguments are validated on the host before anything is launched; on an
  *    error nothing is launched and a vitq_status below is returned.
  *  - Pointers passed to the GEMM / attention paths must be 16-byte aligned.
+ *  - Kernels are launched with programmatic dependent launch: each may start
+ *    while the previous kernel on the stream finishes, and waits for it before
+ *    reading its inputs.  Two reads happen before that wait: LayerNorm's gamma
+ *    and beta (vit_ln_quant, vit_block_forward, the mergers) and attention's
+ *    cu_seqlens (vit_attention_varlen).  So these must not be written by the
+ *    kernel launched immediately before the call on the same stream (weights
+ *    and segment offsets normally are not); otherwise put any stream-ordered
+ *    operation between, or set VITQ_PDL=0 in the environment.
  *
  * Sources (web pages; the section named is where each step is described):
  *  [FRT] "Qwen3-VL-8B on RTX 5090 (NVFP4 language stack + FP8 ViT)"
