@@ -130,8 +130,8 @@ typedef struct {
 
 /* ---------------------------------------------------------------- stages */
 
-/* 1x128 FP8 activation quantisation ([FRT] s3 "per-token / per-128-K-block FP8
- * activation quant"; scale convention [TRT]).  x: bf16 [M, ldx] (first K
+/* 1x128 FP8 activation quantisation ([FRT] s3: activations quantised per token
+ * and per 128-column K block; scale convention [TRT]).  x: bf16 [M, ldx] (first K
  * columns used).  For each row m and K block kb: s = amax / 448 (fp32 IEEE
  * division), q = E4M3_RNE_satfinite(x / s); a zero scale gives zero codes.
  * Outputs q [M, K] and s[kb * lds + m].  K % 16 == 0, lds >= M. */
@@ -155,8 +155,8 @@ int vit_ln_quant(const void* x, int M, int K, int ldx, const void* gamma, const 
  * value, the bf16 rounding of the fp64 value x / (1 + exp(-2u)). */
 int vit_gelu_quant(const void* f, int M, int K, int ldf, uint8_t* q, float* s, int lds, void* stream);
 
-/* FP8 W8A8 block-scaled GEMM with fused bias and residual ([FRT] s1 "FP8
- * block-128 ViT GEMMs", "bias adds fused"; [VE] vision_gemm_bias):
+/* FP8 W8A8 block-scaled GEMM with fused bias and residual ([FRT] s1: the ViT
+ * linears run as FP8 block-128 GEMMs with the bias add fused; [VE] vision_gemm_bias):
  *   C[m,n] = bf16( sum_kb sA[kb*ldsA+m] * sW[(n/128)*ceil(K/128)+kb] * sum_{k in kb} A[m,k] W[n,k]
  *                  + bias[n] + residual[m,n] )
  * A: E4M3 [M, K]; W: E4M3 [N, K]; bias bf16 [N] or NULL; residual bf16 [M, N]
@@ -175,7 +175,7 @@ int fp8_block_gemm(const uint8_t* A, const float* sA, int ldsA, const uint8_t* W
 int bf16_gemm(const void* A, const void* W, const void* bias, const void* residual, void* C, int M, int N, int K,
               void* stream);
 
-/* 2D rotary table ([FRT] s3 "2D rotate_half RoPE"; [VE] rope_inv_freq, head_dim/4
+/* 2D rotary table ([FRT] s3: 2D rotary in rotate_half form; [VE] rope_inv_freq, head_dim/4
  * entries).  pos_hw: int32 [n][2] (row, col) per token.  Output cos_sin fp32
  * [n][72]: cos of the 36 angles then their sines; angle j = row * f_j for
  * j < 18 and col * f_(j-18) otherwise, f_i = theta^(-2i/36).  fp64 inside. */
@@ -202,8 +202,8 @@ int vit_rope2d(void* qkv, int n_tokens, const float* cos_sin, int flags, void* s
 int vit_positions(const int32_t* grid_hw, int n_images, int32_t* pos_hw, int32_t* cu_seqlens,
                   void* stream);
 
-/* Block-diagonal non-causal attention ([FRT] s1/s3 "FA2 (full, bidirectional)",
- * s5 cu_seqlens).  qkv: bf16 [n_tokens, 3, 16, 72] (rotary already applied);
+/* Block-diagonal non-causal attention ([FRT] s1/s3: full, bidirectional
+ * flash attention per block; s5: cu_seqlens).  qkv: bf16 [n_tokens, 3, 16, 72] (rotary already applied);
  * cu_seqlens int32 [n_seqs + 1] with cu[0] = 0, cu[n_seqs] = n_tokens;
  * max_seqlen >= every segment length.  cu_seqlens lives in device memory and
  * is read only by the kernel, so the host cannot check it: it must be
@@ -216,8 +216,8 @@ int vit_positions(const int32_t* grid_hw, int n_images, int32_t* pos_hw, int32_t
 int vit_attention_varlen(const void* qkv, int n_tokens, const int32_t* cu_seqlens, int n_seqs,
                          int max_seqlen, float softmax_scale, int flags, void* out, void* stream);
 
-/* Patch embedding with the interpolated position embedding ([FRT] s3
- * "patch_embed -> +interpolated pos_embed"; [VE] PATCH_DIM = 3*2*16*16 = 1536,
+/* Patch embedding with the interpolated position embedding ([FRT] s3: the
+ * patch embedding is followed by the add of the interpolated position table; [VE] PATCH_DIM = 3*2*16*16 = 1536,
  * patch_embed_w [1152, 1536], pos_embed [2304, 1152], num_grid_per_side 48):
  *   x[t] = bf16( pixels[t] . w^T + b + pos[t] ),
  * pos[t] = bf16(bilinear interpolation of the 48 x 48 table at the token's
@@ -246,7 +246,7 @@ int vit_block_forward(const vitq_block_weights* w, void* x, int n_tokens, const 
                       void* stream);
 size_t vitq_block_workspace_bytes(int n_tokens);
 
-/* 2x2 spatial merger ([FRT] s3 "2x2 patch merger"; [VE] MergerLayer): rows
+/* 2x2 spatial merger ([FRT] s3: the 2x2 merger on each tap; [VE] MergerLayer): rows
  * 4i..4i+3 of x bf16 [n_tokens, 1152] form one 4608 row; LayerNorm(4608)+quant
  * -> fc1 4608->4608 + bias -> GELU+quant -> fc2 4608->2048 + bias.
  * out: bf16 [n_tokens/4, 2048].  n_tokens % 4 == 0. */
@@ -277,8 +277,8 @@ size_t vitq_merger_workspace_bytes(int n_tokens);
 int vit_merger_forward_static(const vitq_merger_weights* w, const void* x, int n_tokens, void* out,
                               void* stream);
 
-/* The 27-block tower over packed images with DeepStack taps ([FRT] s3 "DeepStack
- * taps at layers 8 / 16 / 24", [VE] deepstack_indexes [8,16,24] + final merger).
+/* The 27-block tower over packed images with DeepStack taps ([FRT] s3: DeepStack
+ * taps after layers 8, 16 and 24; [VE] deepstack_indexes [8,16,24] + final merger).
  * x: bf16 [n, 1152] patch embeddings, overwritten with the block-27 output.
  * grid_hw: HOST int32 [n_images][2], every h and w even.  taps[t]: bf16
  * [n/4, 2048] outputs of merger t (after blocks 8, 16, 24, 27).

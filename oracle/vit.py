@@ -155,7 +155,7 @@ def bf16_gemm(a, w, bias=None, residual=None) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
-# LayerNorm and GELU  [FRT s3: "LayerNorm", "GELU(tanh)"; VE norm1_w/b]
+# LayerNorm and GELU  [FRT s3: LayerNorm and GELU(tanh) in the block chain; VE norm1_w/b]
 # --------------------------------------------------------------------------
 
 def layernorm_f64(x, gamma, beta, eps: float = 1e-6) -> np.ndarray:
@@ -201,7 +201,7 @@ def gelu_quant(f) -> tuple:
 
 
 # --------------------------------------------------------------------------
-# Patch order and 2D rotary embedding  [FRT s3 "2D rotate_half RoPE"; VE rope_inv_freq]
+# Patch order and 2D rotary embedding  [FRT s3: 2D rotary in rotate_half form; VE rope_inv_freq]
 # --------------------------------------------------------------------------
 
 def patch_positions(h: int, w: int) -> np.ndarray:
@@ -236,7 +236,7 @@ def packed_positions(grids) -> tuple:
 
 # --------------------------------------------------------------------------
 # Patch embedding and interpolated position embedding
-# [FRT s3 "patch_embed -> +interpolated pos_embed"; VE PATCH_DIM = 3*2*16*16 = 1536,
+# [FRT s3: patch embedding, then the interpolated position table added; VE PATCH_DIM = 3*2*16*16 = 1536,
 #  patch_embed_w [1152, 1536], pos_embed [2304, 1152], num_grid_per_side 48]
 # --------------------------------------------------------------------------
 
@@ -327,7 +327,7 @@ def apply_rope_qkv(qkv, pos, heads: int = 16, head_dim: int = 72, theta: float =
 
 
 # --------------------------------------------------------------------------
-# Block-diagonal non-causal attention  [FRT s1, s3 "FA2 (full, bidirectional)", s5 cu_seqlens]
+# Block-diagonal non-causal attention  [FRT s1, s3: full bidirectional flash attention; s5 cu_seqlens]
 # --------------------------------------------------------------------------
 
 def attention_varlen(qkv, cu_seqlens, heads: int = 16, head_dim: int = 72, scale=None) -> np.ndarray:
