@@ -249,7 +249,8 @@ size_t vitq_block_workspace_bytes(int n_tokens);
 /* 2x2 spatial merger ([FRT] s3: the 2x2 merger on each tap; [VE] MergerLayer): rows
  * 4i..4i+3 of x bf16 [n_tokens, 1152] form one 4608 row; LayerNorm(4608)+quant
  * -> fc1 4608->4608 + bias -> GELU+quant -> fc2 4608->2048 + bias.
- * out: bf16 [n_tokens/4, 2048].  n_tokens % 4 == 0. */
+ * out: bf16 [n_tokens/4, 2048].  n_tokens % 4 == 0.
+ * ws >= vitq_merger_workspace_bytes(n_tokens). */
 int vit_merger_forward(const vitq_merger_weights* w, const void* x, int n_tokens, void* out, void* ws,
                        size_t ws_bytes, void* stream);
 size_t vitq_merger_workspace_bytes(int n_tokens);
@@ -312,8 +313,10 @@ int vit_tower_forward_mixed(const vitq_tower_weights_mixed* w, void* x, const in
 /* ---------------------------------------------------------------- status */
 
 /* Reads and clears the device error word after synchronising `stream`:
- * 0 = none, VITQ_ERR_DEVICE_TIMEOUT = a bounded pipeline wait expired. */
+ * 0 = none, VITQ_ERR_DEVICE_TIMEOUT = a bounded pipeline wait expired,
+ * VITQ_ERR_CUDA if synchronising the stream failed. */
 int vitq_get_device_error(void* stream);
+/* A static English description of a vitq_status ("unknown status" otherwise). */
 const char* vitq_status_string(int status);
 /* Number of kernel launches issued by this library since load (diagnostic). */
 unsigned long long vitq_launch_count(void);

@@ -13,7 +13,7 @@ HEADER = os.path.join(ROOT, "include", "vitq.h")
 def _declared():
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|unsigned long long|char\s*\*|const char\s*\*)\s*\**\s*(\w+)\s*\(",
+    names = re.findall(r"^\s*(?:const\s+)?(?:int|size_t|void|unsigned long long|char\s*\*|const char\s*\*)\s*\**\s*(\w+)\s*\(",
                        src, flags=re.M)
     return sorted(set(names))
 
@@ -139,3 +139,41 @@ def test_size_limits_rejected_on_the_host(built_lib):
     f = lib.vitq_tower_workspace_bytes
     f.restype, f.argtypes = ctypes.c_size_t, [i, i]
     assert f(MAX_ROWS, 4) > 0 and f(MAX_ROWS + 4, 4) == 0
+
+
+_DECL = re.compile(r"^(?:const\s+)?(?:int|size_t|void|char\s*\*|const char\s*\*|unsigned long long)\s*\**\s*(\w+)\s*\(")
+
+
+def _doc_blocks():
+    """(name, the comment block that documents it) for every function the header declares:
+    the comment directly above the declaration, or above a run of declarations (and
+    #defines) that it heads, in which case the block must name the function."""
+    lines = open(HEADER).read().splitlines()
+    out = []
+    for i, ln in enumerate(lines):
+        m = _DECL.match(ln)
+        if not m:
+            continue
+        j, grouped = i - 1, False
+        while j >= 0 and not lines[j].rstrip().endswith("*/"):
+            assert lines[j].startswith(("#define", " ")) or _DECL.match(lines[j]), \
+                f"{m.group(1)}: no comment directly above ({lines[j]!r})"
+            grouped = grouped or bool(_DECL.match(lines[j]))
+            j -= 1
+        k = j
+        while k >= 0 and "/*" not in lines[k]:
+            k -= 1
+        doc = "\n".join(lines[k:j + 1])
+        assert not grouped or m.group(1) in doc, f"{m.group(1)}: shares a comment that does not name it"
+        out.append((m.group(1), doc))
+    return out
+
+
+def test_every_declared_function_is_documented():
+    blocks = _doc_blocks()
+    assert {n for n, _ in blocks} == set(_declared())
+    for name, doc in blocks:
+        assert len(doc) > 40, name
+        if name.startswith("vit_") or name in ("fp8_block_gemm", "bf16_gemm"):
+            # the operation's source section, or a pointer to the entry point that gives it
+            assert re.search(r"\[(FRT|VE|TRT)\]|\bas vit_|merger above|no counterpart", doc), name
