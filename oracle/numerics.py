@@ -81,6 +81,6 @@ def e4m3_encode(v) -> np.ndarray:
 
 
 def bf16_bits_to_f64(bits) -> np.ndarray:
-    """bf16 bit patterns (uint16) to their exact fp64 values."""
+    """bf16 bit patterns (uint16) to their exact fp64 values (bfloat16 format definition)."""
     b = np.asarray(bits, dtype=np.uint32) << 16
     return b.view(np.float32).astype(np.float64)

@@ -82,7 +82,8 @@ def bf16_gemm_fp32(a, w, bias=None, residual=None):
 @contextlib.contextmanager
 def perturbed():
     """Within the context, the oracle's block/merger/tower use the perturbations
-    (fp32 GEMM promotion or accumulation, bf16 attention probabilities)."""
+    (fp32 GEMM promotion or accumulation, bf16 attention probabilities), to measure
+    the depth-growing drift the pages report for FP8 against bf16 [FRT s4]."""
     g, a, b = ov.fp8_block_gemm, ov.attention_varlen, ov.bf16_gemm
     ov.fp8_block_gemm, ov.attention_varlen, ov.bf16_gemm = fp8_block_gemm_fp32_promotion, attention_bf16_p, bf16_gemm_fp32
     try:
