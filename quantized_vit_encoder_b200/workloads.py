@@ -59,8 +59,8 @@ class Workload:
         return self.scales if self.scales else tuple(1.0 for _ in self.grids)
 
 
-# The five workloads.  Config 4's first image is 54x18 (972 patches, the
-# same count as the 36x27 image of config 1) because the 2x2 merger needs an
+# The five workloads.  The packed batch's first image is 54x18 (972 patches,
+# the same count as the single 36x27 image) because the 2x2 merger needs an
 # even grid on both sides.
 WORKLOADS = {
     "block_16x16": Workload("block_16x16", ((16, 16),), 1, False, seed_base=0),
