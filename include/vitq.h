@@ -13,7 +13,11 @@
  *  - The first call on each device that reaches the device checks its
  *    architecture and fills the library's GELU table on that device (a 128 KB
  *    array of the library, one kernel on a private stream, waited for).  Make
- *    that first call before any stream capture begins.
+ *    that first call before any stream capture begins.  This per-device state
+ *    (and the scratch address of vit_merger_forward_static) is kept for the
+ *    life of the process and assumes the device's primary context lives as
+ *    long: after cudaDeviceReset the library's device arrays are gone, so
+ *    the library must not be called again in that process.
  *  - bf16 tensors are passed as `const void*` / `void*` holding IEEE bfloat16
  *    values; FP8 codes are OCP E4M3 ("E4M3FN") bytes; scales are fp32.
  *  - Matrices are row-major.  Activation FP8 codes are [M, K] (K contiguous);
@@ -56,7 +60,8 @@ typedef enum {
   VITQ_ERR_ARCH = 4,          /* current device is not sm_100 */
   VITQ_ERR_CUDA = 5,          /* a CUDA call or kernel launch failed */
   VITQ_ERR_WORKSPACE = 6,     /* workspace smaller than the *_workspace_bytes figure */
-  VITQ_ERR_DEVICE_TIMEOUT = 7 /* a kernel's bounded pipeline wait expired (see vitq_get_device_error) */
+  VITQ_ERR_DEVICE_TIMEOUT = 7, /* a kernel's bounded pipeline wait expired (see vitq_get_device_error) */
+  VITQ_ERR_RANGE = 8           /* a value beyond its storage format was clamped (see vitq_get_device_error) */
 } vitq_status;
 
 /* Model dimensions (Qwen3-VL vision tower: [FRT] section 3, [VE] VisionEncoder). */
@@ -313,8 +318,10 @@ int vit_tower_forward_mixed(const vitq_tower_weights_mixed* w, void* x, const in
 /* ---------------------------------------------------------------- status */
 
 /* Reads and clears the device error word after synchronising `stream`:
- * 0 = none, VITQ_ERR_DEVICE_TIMEOUT = a bounded pipeline wait expired,
- * VITQ_ERR_CUDA if synchronising the stream failed. */
+ * 0 = none, VITQ_ERR_DEVICE_TIMEOUT = a bounded pipeline wait expired (reported
+ * first when both happened), VITQ_ERR_RANGE = a v value beyond +-65504 was
+ * clamped by the fp16 conversion (vit_rope2d with VITQ_V_FP16, the block
+ * paths), VITQ_ERR_CUDA if synchronising the stream failed. */
 int vitq_get_device_error(void* stream);
 /* A static English description of a vitq_status ("unknown status" otherwise). */
 const char* vitq_status_string(int status);

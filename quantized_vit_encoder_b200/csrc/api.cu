@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
@@ -250,6 +251,10 @@ bool merger_weights_ok(const vitq_merger_weights* w) {
          al16(w->norm_w) && al16(w->norm_b);
 }
 
+// Softmax scale 1/sqrt(72), the fp32 value nearest to it (1/sqrtf(72.f) is one ulp
+// below).
+const float kSoftmaxScale = (float)(1.0 / std::sqrt((double)VITQ_HEAD_DIM));
+
 // Algorithmic HBM bytes of the row kernels (read bf16 rows, write codes + scales).
 inline double quant_bytes(double M, double K) { return M * K * 2 + M * K + M * ((K + 127) / 128) * 4; }
 
@@ -271,7 +276,7 @@ int block_impl(const vitq_block_weights* w, __nv_bfloat16* x, int n, const int32
   if (r) return r;
   VITQ_LAUNCH("rope2d", st, 0, dn * 3456 * 2 * 2 + dn * 72 * 4, launch_rope_apply(b.qkv, n, cs, 1, st));
   VITQ_LAUNCH("attention", st, 4.0 * attn_sumsq * VITQ_HEAD_DIM * VITQ_HEADS, dn * VITQ_QKV * 2 + dn * VITQ_HIDDEN * 2,
-              launch_attention(b.qkv, n, cu, n_seqs, max_seqlen, 1.0f / sqrtf((float)VITQ_HEAD_DIM), true, b.attn, st));
+              launch_attention(b.qkv, n, cu, n_seqs, max_seqlen, kSoftmaxScale, true, b.attn, st));
   VITQ_LAUNCH("quant_act", st, 0, quant_bytes(dn, VITQ_HIDDEN),
               launch_quant_act(b.attn, n, VITQ_HIDDEN, VITQ_HIDDEN, b.q, b.s, b.lds, st));
   r = gemm_checked(b.q, b.s, b.lds, w->proj_q, w->proj_s, w->proj_b, x, b.x1, n, VITQ_HIDDEN, VITQ_HIDDEN,
@@ -344,7 +349,7 @@ int block_bf16_impl(const vitq_block_weights_bf16* w, __nv_bfloat16* x, int n, c
   if (r) return r;
   VITQ_LAUNCH("rope2d", st, 0, dn * 3456 * 2 * 2 + dn * 72 * 4, launch_rope_apply(b.qkv, n, cs, 1, st));
   VITQ_LAUNCH("attention", st, 4.0 * attn_sumsq * VITQ_HEAD_DIM * VITQ_HEADS, dn * VITQ_QKV * 2 + dn * VITQ_HIDDEN * 2,
-              launch_attention(b.qkv, n, cu, n_seqs, max_seqlen, 1.0f / sqrtf((float)VITQ_HEAD_DIM), true, b.attn, st));
+              launch_attention(b.qkv, n, cu, n_seqs, max_seqlen, kSoftmaxScale, true, b.attn, st));
   r = bf16_gemm_checked(b.attn, (const bf*)w->proj_w, (const bf*)w->proj_b, x, b.x1, n, VITQ_HIDDEN, VITQ_HIDDEN,
                         num_sms, st);
   if (r) return r;
@@ -799,7 +804,8 @@ int vitq_get_device_error(void* stream) {
   if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v)) != cudaSuccess) return VITQ_ERR_CUDA;
   const unsigned int zero = 0;
   if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return VITQ_ERR_CUDA;
-  return v ? VITQ_ERR_DEVICE_TIMEOUT : VITQ_OK;
+  if (v & kErrWaitTimeout) return VITQ_ERR_DEVICE_TIMEOUT;
+  return v ? VITQ_ERR_RANGE : VITQ_OK;
 }
 
 const char* vitq_status_string(int s) {
@@ -812,6 +818,7 @@ const char* vitq_status_string(int s) {
     case VITQ_ERR_CUDA: return "CUDA error";
     case VITQ_ERR_WORKSPACE: return "workspace too small";
     case VITQ_ERR_DEVICE_TIMEOUT: return "device pipeline wait timed out";
+    case VITQ_ERR_RANGE: return "value beyond the range of its format (clamped)";
     default: return "unknown status";
   }
 }

@@ -466,7 +466,8 @@ __global__ void rope_table_kernel(const int32_t* __restrict__ pos, int n, double
 // x'_j = x_j c_j - x_(j+36) s_j and x'_(j+36) = x_(j+36) c_j + x_j s_j, so no
 // thread reads what another writes.  Items 288..431 are the 8-element chunks of
 // the v heads, converted to fp16 in place when v_to_f16 (round to nearest:
-// exact for 2^-14 <= |v| < 65504, within 2^-25 below).
+// exact for 2^-14 <= |v| <= 65504, within 2^-25 below; larger |v| is clamped to
+// 65504 and flagged in the device error word).
 constexpr int kRopeItems = 432;
 
 __global__ void __launch_bounds__(256) rope_apply_kernel(__nv_bfloat16* __restrict__ qkv,
@@ -499,6 +500,17 @@ __global__ void __launch_bounds__(256) rope_apply_kernel(__nv_bfloat16* __restri
     __nv_bfloat16* dst = base + 2304 + (w - 288) * 8;
     float v[8];
     load8_bf16(dst, v);
+    // fp16 holds |v| <= 65504: larger values are clamped to +-65504 and raise the
+    // range bit of the device error word (NaN passes through unchanged)
+    bool big = false;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (fabsf(v[i]) > 65504.f) {
+        v[i] = copysignf(65504.f, v[i]);
+        big = true;
+      }
+    }
+    if (big) atomicOr(&g_device_error, kErrValueRange);
     __half2 h0 = __floats2half2_rn(v[0], v[1]), h1 = __floats2half2_rn(v[2], v[3]);
     __half2 h2 = __floats2half2_rn(v[4], v[5]), h3 = __floats2half2_rn(v[6], v[7]);
     *reinterpret_cast<uint4*>(dst) = make_uint4(*reinterpret_cast<uint32_t*>(&h0), *reinterpret_cast<uint32_t*>(&h1),

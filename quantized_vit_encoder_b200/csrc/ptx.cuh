@@ -11,9 +11,11 @@ namespace vitq {
 
 // Device-side error word (read and cleared by vitq_get_device_error).  The
 // library is one translation unit, so this is its single definition.
-// Bit values: 1 = a pipeline wait ran past its time limit.
+// Bit values: 1 = a pipeline wait ran past its time limit; 2 = a value did not
+// fit the format it was converted to (v beyond the fp16 range) and was clamped.
 __device__ unsigned int g_device_error = 0;
 constexpr unsigned int kErrWaitTimeout = 1u;
+constexpr unsigned int kErrValueRange = 2u;
 // A wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 // Longest single sleep inside a bounded wait (the abort flag and the limit are
@@ -96,6 +98,27 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t parit
   return ok != 0;
 }
 
+// Non-blocking probe of the phase (returns at once).
+__device__ __forceinline__ bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// How a pipeline wait polls: 0 = try_wait with a suspend-time hint (the warp
+// sleeps until the phase completes or the hint expires), 1 = try_wait without a
+// hint in a loop, 2 = test_wait in a loop.  The limit and the abort flag are
+// checked between sleeps (mode 0) or every 64 polls (modes 1, 2).
+#ifndef VITQ_WAIT_MODE
+#define VITQ_WAIT_MODE 0
+#endif
+
 // Wait for the phase of `bar` with the given parity to complete.  Returns false
 // (and raises the shared abort flag and the device error word) if it has not
 // completed within limit_ns, or if another warp of the CTA already aborted.
@@ -104,13 +127,21 @@ __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, v
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
 #pragma unroll 1
-  while (true) {
+  for (uint32_t n = 0;; ++n) {
+#if VITQ_WAIT_MODE == 0
     if (mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
-    if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > limit_ns) {
-      atomicOr(&g_device_error, kErrWaitTimeout);
-      *abort_flag = 1;
-      return false;
+#elif VITQ_WAIT_MODE == 1
+    if (mbar_try_wait(bar, parity)) return true;
+#else
+    if (mbar_test_wait(bar, parity)) return true;
+#endif
+    if (VITQ_WAIT_MODE == 0 || (n & 63u) == 63u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        atomicOr(&g_device_error, kErrWaitTimeout);
+        *abort_flag = 1;
+        return false;
+      }
     }
   }
 }

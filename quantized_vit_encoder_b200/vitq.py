@@ -18,9 +18,12 @@ LIB_PATH = os.path.join(_HERE, "libvitq.so")
 HIDDEN, HEADS, HEAD_DIM, MLP, QKV = 1152, 16, 72, 4304, 3456
 MERGE_IN, OUT_HIDDEN, N_BLOCKS = 4608, 2048, 27
 PATCH_DIM, POS_GRID = 1536, 48
-STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "pointer not 16-byte aligned",
-          4: "device is not sm_100", 5: "CUDA error", 6: "workspace too small",
-          7: "device pipeline wait timed out"}
+# vitq_status values (include/vitq.h)
+OK, ERR_INVALID_ARG, ERR_SHAPE, ERR_ALIGN, ERR_ARCH, ERR_CUDA, ERR_WORKSPACE, ERR_DEVICE_TIMEOUT, ERR_RANGE = range(9)
+STATUS = {OK: "ok", ERR_INVALID_ARG: "invalid argument", ERR_SHAPE: "unsupported shape",
+          ERR_ALIGN: "pointer not 16-byte aligned", ERR_ARCH: "device is not sm_100", ERR_CUDA: "CUDA error",
+          ERR_WORKSPACE: "workspace too small", ERR_DEVICE_TIMEOUT: "device pipeline wait timed out",
+          ERR_RANGE: "value beyond the range of its format (clamped)"}
 
 _vp, _i, _f, _sz = C.c_void_p, C.c_int, C.c_float, C.c_size_t
 
@@ -187,8 +190,9 @@ def launch_count() -> int:
 
 
 def device_error(stream=None) -> int:
-    """Synchronise the stream, then read and clear the device error word: 0, 7 after a
-    bounded wait timed out, 5 if synchronising failed."""
+    """Synchronise the stream, then read and clear the device error word: OK, ERR_DEVICE_TIMEOUT
+    after a bounded wait timed out, ERR_RANGE after a clamped fp16 v value, ERR_CUDA if
+    synchronising failed."""
     return int(load().vitq_get_device_error(_stream(stream)))
 
 

@@ -44,6 +44,8 @@ def test_host_only_calls(built_lib):
     lib.vitq_status_string.restype = ctypes.c_char_p
     assert lib.vitq_status_string(0) == b"ok"
     assert lib.vitq_status_string(6) == b"workspace too small"
+    assert lib.vitq_status_string(8).startswith(b"value beyond the range")
+    assert lib.vitq_status_string(9) == b"unknown status"
     lib.vitq_block_workspace_bytes.restype = ctypes.c_size_t
     lib.vitq_tower_workspace_bytes.restype = ctypes.c_size_t
     b = lib.vitq_block_workspace_bytes(6256)

@@ -293,7 +293,7 @@ def test_bounded_wait_reports_timeout(lib):
     from quantized_vit_encoder_b200 import vitq
     assert vitq.device_error() == 0
     vitq.selftest_wait_timeout(20000)
-    assert vitq.device_error() == 7
+    assert vitq.device_error() == vitq.ERR_DEVICE_TIMEOUT
     assert vitq.device_error() == 0               # read clears it
     q, s = vitq.quant_act(torch.ones((4, 128), dtype=torch.bfloat16, device="cuda"))
     assert int(q[0, 0]) == 0x7E

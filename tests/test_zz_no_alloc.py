@@ -34,11 +34,11 @@ def test_static_merger_rejects_sizes_beyond_its_scratch():
                    ctypes.c_void_p]
     w = _fake_weights()
     fake = ctypes.c_void_p(4096)
-    assert fn(ctypes.byref(w), fake, MAX_TOKENS + 4, fake, None) == 6   # VITQ_ERR_WORKSPACE
-    assert fn(ctypes.byref(w), fake, 1 << 30, fake, None) == 6
-    assert fn(ctypes.byref(w), fake, 6, fake, None) == 2                # n % 4 != 0
-    assert fn(None, fake, 8, fake, None) == 1
-    assert fn(ctypes.byref(w), None, 8, fake, None) == 1
+    assert fn(ctypes.byref(w), fake, MAX_TOKENS + 4, fake, None) == vitq.ERR_WORKSPACE
+    assert fn(ctypes.byref(w), fake, 1 << 30, fake, None) == vitq.ERR_WORKSPACE
+    assert fn(ctypes.byref(w), fake, 6, fake, None) == vitq.ERR_SHAPE       # n % 4 != 0
+    assert fn(None, fake, 8, fake, None) == vitq.ERR_INVALID_ARG
+    assert fn(ctypes.byref(w), None, 8, fake, None) == vitq.ERR_INVALID_ARG
 
 
 @pytest.mark.gpu
