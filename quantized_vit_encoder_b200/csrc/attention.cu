@@ -13,15 +13,10 @@
 //     combines its row maxima through shared memory).  S_x(j+1) is computed
 //     while the softmax of S_x(j) runs (the softmax frees S_x once it holds it
 //     in registers), and the two tiles interleave on the tensor core;
-//   * the softmax exponentials run on MUFU: with fp16 P (the block's path) as
-//     ex2.approx.f16x2 on the fp16-rounded argument, two results per
-//     instruction, already packed for the P.V operand.  The softmax warps of
-//     tile A and tile B that share an SMSP take turns for their exponentials,
-//     so each turn has MUFU to itself while the other tile reads its next
-//     scores and waits for its P.V;
-//   * row sums come from the tensor core: an otherwise idle warp writes 1 into
-//     V's zero padding column d = 72 of every staged tile, so O column 72
-//     accumulates the row sum of the same rounded P, rescaled with O;
+//   * the softmax exponentials run on MUFU ex2; a share can move to a polynomial
+//     on the FMA pipe (kPolyEvery).  The softmax warps of tile A and tile B that
+//     share an SMSP take turns for their exponentials, so each turn has MUFU to
+//     itself while the other tile reads its next scores and waits for its P.V;
 //   * K and V are read straight from the packed qkv activation [n, 3, 16, 72]
 //     through 3D TMA maps (d, slot, token).  head_dim 72 is padded to 80 by
 //     the tensor map itself: d >= 72 lies outside the map so TMA fills zeros,
@@ -58,9 +53,8 @@ constexpr int kBar = kRed + kQTiles * 2 * 2 * 128 * 4;
 // barriers: slot 0 (unused), kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2],
 // s_free[2], turn[2][4] (the softmax warps of tile x on SMSP q finished their
 // exponentials), q_ready[2] (Q tile x is in TMEM), pair[2][4] (both halves of
-// tile x, quadrant q, posted their partial row maxima), v_ready[S] (the ones
-// column of V stage s is written)
-constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles + kQTiles * 4 + kStages;
+// tile x, quadrant q, posted their partial row maxima)
+constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles + kQTiles * 4;
 constexpr size_t kAttnSmem = 1024 + kBar + kNumBars * 8 + 16;
 static_assert(kAttnSmem <= 232448, "shared memory budget");
 // TMEM columns: S_A 0..127, S_B 128..255, O_A 256..335, Q_A 336..383, O_B 384..463,
@@ -69,9 +63,16 @@ __device__ __forceinline__ uint32_t tmem_s(int x) { return (uint32_t)x * 128u; }
 __device__ __forceinline__ uint32_t tmem_o(int x) { return 256u + (uint32_t)x * 128u; }
 __device__ __forceinline__ uint32_t tmem_q(int x) { return 336u + (uint32_t)x * 128u; }
 // Warpgroup 0: warp 0 TMA producer, warps 1 and 2 MMA issuers for Q tiles A
-// and B, warp 3 writes V's ones column; warps 4-11 softmax of Q tile A, 12-19 of Q tile B (two
+// and B (warp 3 idle); warps 4-11 softmax of Q tile A, 12-19 of Q tile B (two
 // warps per TMEM lane quadrant, each owning 64 of the 128 score columns).
 constexpr int kThreads = 128 + 256 * kQTiles;
+// Share of the softmax exponentials moved from MUFU to the FMA-pipe polynomial:
+// one pair in kPolyEvery (0 = none).  MUFU ex2 runs at 16 per clock per SM.
+#ifndef VITQ_ATTN_POLY_EVERY
+#define VITQ_ATTN_POLY_EVERY 0
+#endif
+constexpr int kPolyEvery = VITQ_ATTN_POLY_EVERY;
+constexpr int kPolyMod = kPolyEvery > 0 ? kPolyEvery : 1;
 // 8-key group of the exponential loop after which the turn passes to the other tile (7 = at the end).
 #ifndef VITQ_ATTN_TURN_AT
 #define VITQ_ATTN_TURN_AT 5
@@ -118,9 +119,6 @@ struct AttnSmem {
   __device__ uint32_t pair(int x, int q) const {
     return smem_u32(bar(1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles + x * 4 + q));
   }
-  __device__ uint32_t v_ready(int s) const {
-    return smem_u32(bar(1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles + kQTiles * 4 + s));
-  }
   __device__ float* red(int x, int par, int h) const {
     return reinterpret_cast<float*>(base + kRed) + ((x * 2 + par) * 2 + h) * 128;
   }
@@ -137,6 +135,27 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+
+// 2^x on the FMA/ALU pipes for a pair of values (Cody-Waite split x = n + f,
+// |f| <= 1/2, then a degree-3 polynomial fitted to 2^f on [-1/2, 1/2]: max
+// relative error 7.5e-5, below the fp16 rounding of P).  n is read from the low
+// bits of x + 1.5*2^23 and added to the exponent field; x is clamped at -125
+// (2^-125 is 0 once P is rounded).
+// ex2_poly on a pair of values with packed fp32 arithmetic.
+__device__ __forceinline__ float2 ex2_poly2(float x0, float x1) {
+  const uint64_t magic = f2pack(12582912.0f, 12582912.0f), nmagic = f2pack(-12582912.0f, -12582912.0f);
+  const uint64_t x = f2pack(fmaxf(x0, -125.0f), fmaxf(x1, -125.0f));
+  const uint64_t j = fadd2(x, magic);
+  const uint64_t f = ffma2(fadd2(j, nmagic), f2pack(-1.0f, -1.0f), x);
+  uint64_t p = ffma2(f2pack(0.0551716648f, 0.0551716648f), f, f2pack(0.2426111251f, 0.2426111251f));
+  p = ffma2(p, f, f2pack(0.6932609677f, 0.6932609677f));
+  p = ffma2(p, f, f2pack(0.9999280572f, 0.9999280572f));
+  const float2 pp = f2unpack(p), jj = f2unpack(j);
+  return make_float2(__int_as_float(__float_as_int(pp.x) + (__float_as_int(jj.x) << 23)),
+                     __int_as_float(__float_as_int(pp.y) + (__float_as_int(jj.y) << 23)));
+}
+
+
 
 __device__ void attn_producer(const AttnSmem& sm, const CUtensorMap* tlo, const CUtensorMap* thi,
                               int head, int kv_row0, int n_kv, int off) {
@@ -175,11 +194,10 @@ template <bool kVF16>
 __device__ bool attn_issue_pv(const AttnSmem& sm, uint32_t tmem, int x, int j) {
   constexpr uint32_t fmt = kVF16 ? 0u : 1u;
   constexpr uint32_t idesc = make_idesc(fmt, fmt, 0, 1, 128, 80);
-  const int s = j % kStages;
-  if (!mbar_wait(sm.v_ready(s), (uint32_t)(j / kStages) & 1u, sm.abort_flag())) return false;
   if (!mbar_wait(sm.p_full(x), (uint32_t)j & 1u, sm.abort_flag())) return false;
   VITQ_TRACE_EV(14 + x, j);   // mma: P complete
   tc_fence_after();
+  const int s = j % kStages;
   const uint32_t vlo = sm.kv(s, kVLo), p0 = sm.p(x);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
@@ -215,41 +233,12 @@ __device__ void attn_mma(const AttnSmem& sm, uint32_t tmem, int x, int n_kv) {
   }
 }
 
-// Row sums from the tensor core: V's padding column d = 72 (zero-filled by TMA)
-// is set to 1 in every staged V tile, so O column 72 accumulates the sum of the
-// same rounded P the numerator uses, rescaled with it.  One warp writes the 128
-// keys' d 72..79 chunk of the V hi tile (1, 0, ..., 0) once the stage has landed.
-template <bool kVF16>
-__device__ void attn_ones_writer(const AttnSmem& sm, int n_kv) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t one = kVF16 ? 0x3C00u : 0x3F80u;   // 1.0 in fp16 / bf16, element d = 72
-  for (int j = 0; j < n_kv; ++j) {
-    const int s = j % kStages;
-    const bool ok = mbar_wait(sm.kv_full(s), (uint32_t)(j / kStages) & 1u, sm.abort_flag());
-    if (!__all_sync(0xffffffffu, ok)) return;
-    uint8_t* vhi = sm.base + kKV0 + s * kKVStride + kVHi;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int r = lane + 32 * i;   // key row; chunk 1 of its 128-byte row holds d 72..79
-      *reinterpret_cast<uint4*>(vhi + r * 128 + ((1 ^ (r & 7)) << 4)) = make_uint4(one, 0u, 0u, 0u);
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sm.v_ready(s));
+__device__ __forceinline__ uint32_t pack_p(float lo, float hi, bool f16) {
+  if (f16) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
   }
-}
-
-// fp32 pair -> f16x2 (lo in bits 0..15), round to nearest even
-__device__ __forceinline__ uint32_t f16x2_of(float lo, float hi) {
-  uint32_t w;
-  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(w) : "f"(hi), "f"(lo));
-  return w;
-}
-// 2^x on both halves of an f16x2 (one MUFU instruction for two results)
-__device__ __forceinline__ uint32_t ex2_f16x2(uint32_t x) {
-  uint32_t y;
-  asm("ex2.approx.f16x2 %0, %1;" : "=r"(y) : "r"(x));
-  return y;
+  return pack_bf16x2(lo, hi);
 }
 
 // Two warps per (Q tile, TMEM lane quadrant); thread = query row = TMEM lane.
@@ -291,7 +280,7 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.q_ready(x));
   }
-  float m_run = -INFINITY;
+  float m_run = -INFINITY, l_run = 0.f;
   for (int j = 0; j < n_kv; ++j) {
     bool ok = mbar_wait(sm.s_full(x), (uint32_t)j & 1u, sm.abort_flag());
     if (!__all_sync(0xffffffffu, ok)) return;
@@ -361,10 +350,9 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
     }
     if (tr) VITQ_TRACE_EV(28 + x, j);   // softmax: turn for the exponentials
     // P = 2^(s * scale_log2 - m_run), rounded to the P.V operand type, into this
-    // half's 64-key atom of the swizzled P tile.  fp16 P: the exponent argument is
-    // rounded to fp16 and ex2.approx.f16x2 gives two P values in one MUFU
-    // instruction, already packed; bf16 P: fp32 ex2 and a packing conversion.
+    // half's 64-key atom of the swizzled P tile; 8 fp32 partial row sums.
     const uint64_t sc2 = f2pack(g.scale_log2, g.scale_log2), nm2 = f2pack(-m_run, -m_run);
+    uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
       uint32_t w[4];
@@ -374,10 +362,16 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
         const float2 t = f2unpack(ffma2(f2pack(__uint_as_float(su[k0 >> 5][k0 & 31]),
                                                __uint_as_float(su[(k0 + 1) >> 5][(k0 + 1) & 31])),
                                         sc2, nm2));
-        if (kVF16)
-          w[i] = ex2_f16x2(f16x2_of(t.x, t.y));
-        else
-          w[i] = pack_bf16x2(ex2(t.x), ex2(t.y));
+        // every kPolyEvery-th pair runs the FMA-pipe polynomial, the rest MUFU ex2
+        float2 p;
+        if (kPolyEvery > 0 && (i % kPolyMod) == kPolyMod - 1) {
+          p = ex2_poly2(t.x, t.y);
+        } else {
+          p.x = ex2(t.x);
+          p.y = ex2(t.y);
+        }
+        w[i] = pack_p(p.x, p.y, kVF16);
+        ls[i] = fadd2(ls[i], f2pack(p.x, p.y));
       }
       uint8_t* dst = pbase + r * 128 + ((c ^ (r & 7)) << 4);
       *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
@@ -401,34 +395,36 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
       }
       tmem_wait_st();
     }
+    {
+      const float2 l0 = f2unpack(fadd2(ls[0], ls[1])), l1 = f2unpack(fadd2(ls[2], ls[3]));
+      l_run = l_run * alpha + ((l0.x + l0.y) + (l1.x + l1.y));
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncwarp();
     if (tr) VITQ_TRACE_EV(24 + x, j);   // softmax: P written
     if (lane == 0) mbar_arrive(sm.p_full(x));
   }
-  if (h != 0) return;
   bool ok = mbar_wait(sm.pv_done(x), (uint32_t)(n_kv - 1) & 1u, sm.abort_flag());
   if (!__all_sync(0xffffffffu, ok)) return;
   tc_fence_after();
-  // the row sum is O's column 72 (the ones column of V); O / l in 16-column chunks
-  // (columns 72..79 are not stored)
-  uint32_t u4[16];
-  tmem_ld16(o_addr + 64, u4);
-  tmem_wait_ld();
+  // row sum = the two halves' partial sums (one more exchange, slot parity n_kv)
+  sm.red(x, n_kv & 1, h)[r] = l_run;
+  __syncwarp();
+  if (lane == 0) mbar_arrive(sm.pair(x, quad));
+  ok = mbar_wait(sm.pair(x, quad), (uint32_t)n_kv & 1u, sm.abort_flag());
+  if (!__all_sync(0xffffffffu, ok)) return;
+  if (h != 0) return;
+  const float l_sum = l_run + sm.red(x, n_kv & 1, 1)[r];
+  // O / l in 16-column chunks (columns 72..79 are the zero padding and are not stored)
   const bool row_ok = q0 + r < seq_len && seq_start + q0 + r < g.n_tokens;
-  const float inv = 1.0f / __uint_as_float(u4[8]);
+  const float inv = 1.0f / l_sum;
   __nv_bfloat16* dst = g.out + (size_t)(seq_start + q0 + r) * 1152 + head * 72;
 #pragma unroll
   for (int c = 0; c < 5; ++c) {
     uint32_t u[16];
-    if (c < 4) {
-      tmem_ld16(o_addr + c * 16, u);
-      tmem_wait_ld();
-    } else {
-#pragma unroll
-      for (int i = 0; i < 16; ++i) u[i] = u4[i];
-    }
+    tmem_ld16(o_addr + c * 16, u);
+    tmem_wait_ld();
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       if (row_ok && c * 2 + hh < 9) {
@@ -464,7 +460,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(sm.kv_full(s), 1);
       mbar_init(sm.kv_empty(s), (uint32_t)n_q);       // one commit per active Q tile
-      mbar_init(sm.v_ready(s), 1);
     }
     for (int x = 0; x < kQTiles; ++x) {
       for (int q = 0; q < 4; ++q) mbar_init(sm.turn(x, q), 2);
@@ -494,8 +489,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       attn_producer(sm, &tlo, &thi, head, seq_start, n_kv, off);
     } else if ((warp == 1 || warp == 2) && lane == 0 && warp - 1 < n_q) {
       attn_mma<kVF16>(sm, tmem, warp - 1, n_kv);
-    } else if (warp == 3) {
-      attn_ones_writer<kVF16>(sm, n_kv);
     }
   } else {
     const int x = (warp - 4) >> 3, h = ((warp - 4) >> 2) & 1;

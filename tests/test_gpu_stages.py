@@ -285,17 +285,18 @@ def test_rope_v_fp16_range_guard(lib):
     qkv[3, 2304 + 5] = 1.0e5
     qkv[3, 2304 + 6] = -3.0e38
     qkv[5, 2304 + 100] = float("nan")
-    qkv[6, 2304 + 7] = 65504.0
+    qkv[6, 2304 + 7] = 65536.0        # bf16 has no 65504: the nearest values are 65280 and 65536
+    qkv[6, 2304 + 8] = 65280.0        # in range: kept exactly
     assert vitq.device_error() == vitq.OK
     got = vitq.rope2d_(qkv.cuda().clone(), cs, flags=vitq.V_FP16)
     assert vitq.device_error() == vitq.ERR_RANGE
     assert vitq.device_error() == vitq.OK
     v16 = got[:, 2304:].contiguous().view(torch.float16).float().cpu()
     v = qkv[:, 2304:].float()
-    assert v16[3, 5] == 65504.0 and v16[3, 6] == -65504.0 and v16[6, 7] == 65504.0
+    assert v16[3, 5] == 65504.0 and v16[3, 6] == -65504.0 and v16[6, 7] == 65504.0 and v16[6, 8] == 65280.0
     assert torch.isnan(v16[5, 100])
     keep = torch.ones_like(v, dtype=torch.bool)
-    keep[3, 5] = keep[3, 6] = keep[5, 100] = False
+    keep[3, 5] = keep[3, 6] = keep[5, 100] = keep[6, 7] = False
     assert torch.equal(v16[keep], v.half().float()[keep])
     # no flag when everything fits
     vitq.rope2d_(bf16((8, 3456), 72, 1.0).cuda(), cs, flags=vitq.V_FP16)
