@@ -54,19 +54,23 @@ def _table():
 
 
 def test_roofline_of_the_dominant_kernel():
-    peaks = {"hbm_gbs": 6455.6, "bf16": 1649.5, "bf16_sustained": 1415.6, "source": "measured"}
+    peaks = {"hbm_gbs": 6455.6, "bf16": 1649.5, "bf16_sustained": 1415.6, "source": "measured",
+             "fp8": 3300.0, "fp8_sustained": 2900.0, "fp8_source": "measured"}
     r = bench.roofline(_table(), peaks)
     per_launch_s = 15.34e-3 / 54
     assert r["kernel"] == "attention" and r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert abs(r["achieved"] - 180.35e9 / per_launch_s / 1e12) < 1e-9
-    assert r["peak"] == 1415.6 and abs(r["frac"] - r["achieved"] / 1415.6) < 1e-12
+    # the burst peak (kernels timed inside a short step), the sustained one as context
+    assert r["peak"] == 1649.5 and abs(r["frac"] - r["achieved"] / 1649.5) < 1e-12
+    assert r["sustained_peak"] == 1415.6 and abs(r["frac_of_sustained"] - r["achieved"] / 1415.6) < 1e-12
     assert r["nominal_peak"] == 2250.0 and abs(r["frac_of_nominal"] - r["achieved"] / 2250.0) < 1e-12
     assert abs(r["share"] - 15.34 / (15.34 + 10.48 + 3.31)) < 1e-12
-    # a GEMM-dominated table takes the FP8 peak (measured bf16 x 2), an HBM-bound one GB/s
+    # a GEMM-dominated table takes the measured FP8 peak, an HBM-bound one GB/s
     t = _table()
     t["fp8_block_gemm"]["ms"] = 40.0
     g = bench.roofline(t, peaks)
-    assert g["kernel"] == "fp8_block_gemm" and g["peak"] == 2 * 1415.6 and g["nominal_peak"] == 4500.0
+    assert g["kernel"] == "fp8_block_gemm" and g["peak"] == 3300.0 and g["nominal_peak"] == 4500.0
+    assert bench.load_peaks()["fp8"] == 2 * bench.load_peaks()["bf16"]     # before the FP8 measurement
     t["ln_quant"]["ms"] = 100.0
     h = bench.roofline(t, peaks)
     assert h["bound"] == "hbm" and h["unit"] == "GB/s" and h["peak"] == 6455.6
