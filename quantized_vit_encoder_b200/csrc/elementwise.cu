@@ -292,8 +292,9 @@ __global__ void __launch_bounds__(16 * kLnRows, 6)
       slow |= (uint32_t)(lo != hi) << i;
       w[i] = lo;
     }
-    if (slow) {   // rare (about 2^-11 of the pairs): those pairs in fp64
-#pragma unroll 1
+    if (slow) {   // rare (about 2^-11 of the pairs): those pairs in fp64 (unrolled: a
+                  // runtime index would put v, g, b and w in local memory for every chunk)
+#pragma unroll
       for (int i = 0; i < 4; ++i)
         if ((slow >> i) & 1u)
           w[i] = ln_pair_fp64(v[2 * i], v[2 * i + 1], g[2 * i], g[2 * i + 1], b[2 * i], b[2 * i + 1], mean, rstd);
