@@ -60,8 +60,11 @@ struct GemmCfg {
   static constexpr int MIN_LAUNCH_REGS = 168;   // 384 x 168 >= 128 x 56 + 256 x 224 (BN = 256)
   static constexpr int OUT_WARP_BYTES = NH * 4096;  // 64-column SW128 boxes of 32 rows
   static constexpr int OUT_BYTES = EPI_WARPS * (OUT_WARP_BYTES + COLS * 2);   // + the warp's bias values
+  // per epilogue warp, its 32 rows' activation scales of the next SA_DEPTH K blocks
+  static constexpr int SA_DEPTH = 8;
+  static constexpr int SA_BYTES = EPI_WARPS * SA_DEPTH * 32 * 4;
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF + EPI_WARPS) * 8 + 16;
-  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + OUT_BYTES + 1024 + BAR_BYTES;
+  static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + OUT_BYTES + SA_BYTES + 1024 + BAR_BYTES;
 };
 static_assert(384 * GemmCfg<256>::MIN_LAUNCH_REGS >= 128 * 56 + 256 * 224, "register split");
 
@@ -90,8 +93,12 @@ struct GemmSmem {
     return base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + (size_t)Cfg::EPI_WARPS * Cfg::OUT_WARP_BYTES +
            w * Cfg::COLS * 2;
   }
+  __device__ uint32_t sa_ring(int w) const {
+    return smem_u32(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES + w * Cfg::SA_DEPTH * 128);
+  }
   __device__ uint64_t* bars() const {
-    return reinterpret_cast<uint64_t*>(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES);
+    return reinterpret_cast<uint64_t*>(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES +
+                                       Cfg::SA_BYTES);
   }
   __device__ uint32_t full(int s) const { return smem_u32(bars() + s); }
   __device__ uint32_t empty(int s) const { return smem_u32(bars() + Cfg::STAGES + s); }
@@ -212,16 +219,44 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
   const bool has_res = g.residual != nullptr;
   // the leader's tempty barriers count both CTAs' epilogue warps
   const uint32_t tempty0 = kPair ? mapa_shared(sm.tempty(0), 0) : sm.tempty(0);
+  // Activation scales run SA_DEPTH - 1 K blocks ahead of their use through a ring
+  // of SA_DEPTH slots in shared memory: each lane copies its own row's scale
+  // (cp.async, zero past M), one group per K block, continuing into the next
+  // tile's first K blocks, so a warp that falls behind the MMAs never waits for a
+  // scale from L2.  A copy goes into the slot read one K block earlier.
+  const uint32_t ring = sm.sa_ring(ew) + lane * 4;
+  int pf_tile = t0, pf_kb = 0, pf_row = 0;
+  auto pf_row_of = [&](int tile) {
+    int mt_, nt_;
+    tile_coords(tile, tiles_m, tiles_n, mt_, nt_);
+    return mt_ * Cfg::TILE_M + rank * Cfg::BM + r_in;
+  };
+  if (pf_tile < num_tiles) pf_row = pf_row_of(pf_tile);
+  uint32_t pf_q = 0;
+  auto prefetch_scale = [&]() {
+    if (pf_tile < num_tiles) {
+      const bool in = pf_row < g.M;
+      cp_async4(ring + (pf_q & (Cfg::SA_DEPTH - 1)) * 128, in ? g.sA + (size_t)pf_kb * g.ldsA + pf_row : g.sA,
+                in ? 4u : 0u);
+      if (++pf_kb == nkb) {
+        pf_kb = 0;
+        pf_tile += dt;
+        if (pf_tile < num_tiles) pf_row = pf_row_of(pf_tile);
+      }
+    }
+    cp_async_commit();
+    ++pf_q;
+  };
+#pragma unroll 1
+  for (int i = 0; i < Cfg::SA_DEPTH - 1; ++i) prefetch_scale();
   uint32_t cnt = 0, it = 0;
   for (int tile = t0; tile < num_tiles; tile += dt, ++it) {
     int mt, nt;
     tile_coords(tile, tiles_m, tiles_n, mt, nt);
     const int m0 = mt * Cfg::TILE_M + rank * Cfg::BM;
     const int n0 = nt * BN;
-    const int row = m0 + r_in;
     const int col0 = n0 + cg * Cfg::COLS;
     const int y0 = m0 + quad * 32;                   // first row of this warp's staging tile
-    const bool row_ok = row < g.M;
     const bool col_ok = col0 < g.N;
     // this warp's COLS bias values (lane l: columns 4l..4l+3), loaded now and
     // parked in shared memory after the K loop
@@ -239,22 +274,19 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
       }
       __syncwarp();
     }
-    const float* sa_ptr = g.sA + row;
     const float* sw_ptr = g.sW + (size_t)(col0 >> 7) * nkb;
     uint64_t acc[Cfg::NH * 32];
 #pragma unroll
     for (int j = 0; j < Cfg::NH * 32; ++j) acc[j] = 0ull;
-    // scales are loaded one K block ahead so their latency hides behind the previous block
-    float sa_next = row_ok ? __ldg(sa_ptr) : 0.f;
+    // the weight scale (the same for the whole warp, an L1 hit) is loaded one K block ahead
     float sw_next = col_ok ? __ldg(sw_ptr) : 0.f;
     for (int kb = 0; kb < nkb; ++kb, ++cnt) {
       const uint32_t buf = cnt % Cfg::NBUF;
       const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
-      const float scale = sa_next * sw_next;
-      if (kb + 1 < nkb) {
-        sa_next = row_ok ? __ldg(sa_ptr + (size_t)(kb + 1) * g.ldsA) : 0.f;
-        sw_next = col_ok ? __ldg(sw_ptr + kb + 1) : 0.f;
-      }
+      cp_async_wait<Cfg::SA_DEPTH - 2>();
+      const float scale = ld_shared_f32(ring + (cnt & (Cfg::SA_DEPTH - 1)) * 128) * sw_next;
+      prefetch_scale();
+      if (kb + 1 < nkb) sw_next = col_ok ? __ldg(sw_ptr + kb + 1) : 0.f;
       const uint64_t s2 = f2pack(scale, scale);
       if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(4, cnt);  // epilogue: waiting for partial
       const bool ok = mbar_wait(sm.tfull(buf), aph, sm.abort_flag());
@@ -268,6 +300,19 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
         tmem_ld32(taddr + h * 64, r0);
         tmem_ld32(taddr + h * 64 + 32, r1);
         tmem_wait_ld();
+        if (h == Cfg::NH - 1) {
+          // the whole partial is in registers: the buffer goes back to the MMA
+          // thread before the last FMAs, which keeps them off the hand-off chain
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(6, cnt);  // epilogue: partial consumed
+          if (lane == 0) {
+            if (kPair)
+              mbar_arrive_cluster(tempty0 + buf * 8);
+            else
+              mbar_arrive(sm.tempty(buf));
+          }
+        }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           acc[h * 32 + j] = ffma2(f2pack(__uint_as_float(r0[2 * j]), __uint_as_float(r0[2 * j + 1])), s2,
@@ -275,15 +320,6 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
           acc[h * 32 + 16 + j] = ffma2(f2pack(__uint_as_float(r1[2 * j]), __uint_as_float(r1[2 * j + 1])), s2,
                                       acc[h * 32 + 16 + j]);
         }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(6, cnt);  // epilogue: partial consumed
-      if (lane == 0) {
-        if (kPair)
-          mbar_arrive_cluster(tempty0 + buf * 8);
-        else
-          mbar_arrive(sm.tempty(buf));
       }
     }
     if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(7, it);  // epilogue: K loop done
