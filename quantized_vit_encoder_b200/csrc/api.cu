@@ -107,15 +107,21 @@ int cuda_status(cudaError_t e) {
 int pick_block_n(int M, int N, int num_sms) {
   if (const char* env = std::getenv("VITQ_GEMM_BN")) {
     const int v = std::atoi(env);
-    if (v == 128 || v == 256) return v;
+    if (v == 64 || v == 128 || v == 256) return v;
   }
-  // Every 128-wide K block of a tile costs a fixed ~450-500 cycles beyond its MMA
-  // work (measured), so 128 x 256 tiles, with half as many K blocks per output,
-  // win where N is wide; narrow outputs keep 128 for enough tiles per SM (and
-  // four TMEM partial buffers, which hide the epilogue).
-  (void)M;
-  (void)num_sms;
-  return N > 1536 ? 256 : 128;
+  // Every 128-wide K block of a tile costs a fixed ~580 cycles of MMA issue
+  // whatever the tile width (measured), so 128 x 256 tiles, with half as many K
+  // blocks per output, win where N is wide and M fills the GPU; narrow outputs
+  // keep 128 for enough tiles per SM (and four TMEM partial buffers, which hide
+  // the epilogue).  Where the narrower tiling still leaves half of the SMs free
+  // (small M), it runs each tile sooner and on more SMs; a narrower tiling that
+  // fills the GPU measured slower in the block (the next kernel, launched early,
+  // finds no free SM to start on).  Each output element is computed the same way
+  // at every tile width, so the choice does not change results.
+  const long long tiles_m = (M + 127) / 128;
+  const long long half = num_sms / 2;
+  if (N > 1536) return tiles_m * ((N + 127) / 128) <= half ? 128 : 256;
+  return tiles_m * ((N + 63) / 64) <= half ? 64 : 128;
 }
 
 // Workspace carving helper.

@@ -34,6 +34,7 @@
 namespace vitq {
 namespace {
 
+// BN = 64: 6 warps (TMA, MMA, 4 epilogue warps, one per 32 rows); for small M.
 // BN = 128: 10 warps (TMA, MMA, 8 epilogue warps, one per 64 columns x 32 rows).
 // BN = 256: 12 warps
 // (warpgroup 0 = TMA, MMA and two idle warps, which give registers away with
@@ -43,14 +44,14 @@ struct GemmCfg {
   static constexpr int BM = 128, BK = 128;            // rows of A per CTA, K per stage
   static constexpr int TILE_M = kPair ? 256 : 128;    // rows per output tile
   static constexpr int B_ROWS = kPair ? BN / 2 : BN;  // rows of W loaded per CTA
-  static constexpr int STAGES = kPair ? (BN == 256 ? 4 : 7) : (BN == 256 ? 3 : 5);
+  static constexpr int STAGES = kPair ? (BN == 256 ? 4 : 7) : (BN == 256 ? 3 : BN == 128 ? 5 : 7);
   static constexpr int A_BYTES = BM * BK;
   static constexpr int B_BYTES = B_ROWS * BK;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int NBUF = 512 / BN;
-  // columns per epilogue warp: 64 for BN = 128 (8 epilogue warps: one TMEM round
-  // trip per K block each), 128 for BN = 256 (the register file holds no more)
-  static constexpr int COLS = BN == 128 ? 64 : 128;
+  // columns per epilogue warp: 64 for BN = 64 / 128 (4 / 8 epilogue warps: one TMEM
+  // round trip per K block each), 128 for BN = 256 (the register file holds no more)
+  static constexpr int COLS = BN == 256 ? 128 : 64;
   static constexpr int NH = COLS / 64;                // 64-column halves per warp
   static constexpr int EPI_WARPS = (BN / COLS) * 4;
   static constexpr int TEMPTY_COUNT = EPI_WARPS * (kPair ? 2 : 1);   // both CTAs' epilogues free a buffer
@@ -516,7 +517,7 @@ cudaError_t launch_fp8_gemm(const uint8_t* A, const float* sA, int ldsA, const u
                             int M, int N, int K, int block_n, bool pair, int num_sms, cudaStream_t st) {
   if (M == 0 || N == 0) return cudaSuccess;
   CUtensorMap tmA, tmB, tmC, tmR;
-  const int bn = block_n == 256 ? 256 : 128;
+  const int bn = block_n == 256 ? 256 : (block_n == 64 && !pair) ? 64 : 128;
   cudaError_t e = encode_tma_2d_u8(&tmA, A, K, M, 128, 128);
   if (e != cudaSuccess) return e;
   e = encode_tma_2d_u8(&tmB, W, K, N, 128, pair ? bn / 2 : bn);
@@ -529,6 +530,7 @@ cudaError_t launch_fp8_gemm(const uint8_t* A, const float* sA, int ldsA, const u
   if (pair)
     return bn == 256 ? launch_bn<256, true>(tmA, tmB, tmC, tmR, a, num_sms, st)
                      : launch_bn<128, true>(tmA, tmB, tmC, tmR, a, num_sms, st);
+  if (bn == 64) return launch_bn<64, false>(tmA, tmB, tmC, tmR, a, num_sms, st);
   return bn == 256 ? launch_bn<256, false>(tmA, tmB, tmC, tmR, a, num_sms, st)
                    : launch_bn<128, false>(tmA, tmB, tmC, tmR, a, num_sms, st);
 }

@@ -175,10 +175,11 @@ GEMM_SHAPES = [
 
 
 @pytest.mark.parametrize("pair", [0, 1], ids=["cta", "pair"])
-@pytest.mark.parametrize("bn", [128, 256])
+@pytest.mark.parametrize("bn", [64, 128, 256])
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
 def test_fp8_gemm_matches_oracle(lib, monkeypatch, pair, bn, M, N, K):
-    """One CTA per tile and CTA pairs (cta_group::2 MMA over 256-row tiles)."""
+    """One CTA per tile and CTA pairs (cta_group::2 MMA over 256-row tiles; pairs run
+    64-wide requests as 128)."""
     from quantized_vit_encoder_b200 import vitq
     monkeypatch.setenv("VITQ_GEMM_BN", str(bn))
     monkeypatch.setenv("VITQ_GEMM_PAIR", str(pair))
@@ -200,6 +201,29 @@ def test_fp8_gemm_matches_oracle(lib, monkeypatch, pair, bn, M, N, K):
     assert_close(got, ref, what=f"gemm {M}x{N}x{K} bn{bn} pair{pair}")
     # the promotion is fp32 against an fp64 oracle: nearly every bf16 output is identical
     assert np.mean(got == ref) > 0.97
+
+
+@pytest.mark.parametrize("M,N,K,res", [(256, 3456, 1152, False), (300, 1152, 4304, True),
+                                       (972, 4304, 1152, False), (6256, 1152, 1152, True)])
+def test_fp8_gemm_tile_width_invariant(lib, monkeypatch, M, N, K, res):
+    """Every tile width gives the same bits: each output element is the same chain of
+    per-K-block FMAs whatever the tile, so the library may pick the width from M (more,
+    narrower tiles for small M) without making a packed batch differ from its images."""
+    from quantized_vit_encoder_b200 import vitq
+    a = bf16((M, K), 80 + M, 1.0)
+    w = bf16((N, K), 81 + N, 0.02)
+    bias = bf16((N,), 82, 0.01).cuda()
+    r = bf16((M, N), 83, 1.0).cuda() if res else None
+    qa, sa = vitq.quant_act(a.cuda())
+    qw, sw = vitq.quant_weight(w.cuda())
+    outs = []
+    for bn in (64, 128, 256):
+        monkeypatch.setenv("VITQ_GEMM_BN", str(bn))
+        outs.append(vitq.fp8_block_gemm(qa, sa, qw, sw, bias, r).view(torch.int16).cpu())
+    monkeypatch.delenv("VITQ_GEMM_BN")
+    outs.append(vitq.fp8_block_gemm(qa, sa, qw, sw, bias, r).view(torch.int16).cpu())   # the library's pick
+    for o in outs[1:]:
+        assert torch.equal(o, outs[0])
 
 
 BF16_GEMM_SHAPES = [
