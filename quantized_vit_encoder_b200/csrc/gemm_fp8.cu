@@ -61,9 +61,13 @@ struct GemmCfg {
   static constexpr int MIN_LAUNCH_REGS = 168;   // 384 x 168 >= 128 x 56 + 256 x 224 (BN = 256)
   static constexpr int OUT_WARP_BYTES = NH * 4096;  // 64-column SW128 boxes of 32 rows
   static constexpr int OUT_BYTES = EPI_WARPS * (OUT_WARP_BYTES + COLS * 2);   // + the warp's bias values
-  // per epilogue warp, its 32 rows' activation scales of the next SA_DEPTH K blocks
+  // BN = 256 (single CTAs): warp 2, otherwise idle, stages each K block's combined
+  // scales sA * sW for the tile's 128 rows and two weight blocks in a slot tied to
+  // the K block's TMEM buffer.  Otherwise each epilogue warp keeps its 32 rows'
+  // activation scales of the next SA_DEPTH K blocks in its own ring.
+  static constexpr bool SCALE_WARP = BN == 256 && !kPair;
   static constexpr int SA_DEPTH = 8;
-  static constexpr int SA_BYTES = EPI_WARPS * SA_DEPTH * 32 * 4;
+  static constexpr int SA_BYTES = SCALE_WARP ? NBUF * 2 * 128 * 4 : EPI_WARPS * SA_DEPTH * 32 * 4;
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF + EPI_WARPS) * 8 + 16;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + OUT_BYTES + SA_BYTES + 1024 + BAR_BYTES;
 };
@@ -93,6 +97,10 @@ struct GemmSmem {
   __device__ uint8_t* bias(int w) const {
     return base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + (size_t)Cfg::EPI_WARPS * Cfg::OUT_WARP_BYTES +
            w * Cfg::COLS * 2;
+  }
+  // combined scales of TMEM buffer b, weight block cb of the tile (128 rows, fp32)
+  __device__ uint32_t scale_slot(int b, int cb) const {
+    return smem_u32(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES + (b * 2 + cb) * 512);
   }
   __device__ uint32_t sa_ring(int w) const {
     return smem_u32(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES + w * Cfg::SA_DEPTH * 128);
@@ -205,6 +213,56 @@ __device__ void gemm_mma(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base, int 
   }
 }
 
+// Scale producer (BN = 256): for each K block of this CTA's tiles, in the MMA's
+// order, sA[kb, m] * sW[n / 128, kb] for the tile's 128 rows and both weight blocks
+// into the slot of the K block's TMEM buffer, once the epilogue has released that
+// buffer (the tempty phase the MMA thread waits for); then one arrival on the
+// buffer's tfull barrier, which completes when this and the MMAs' commit have both
+// arrived.  Lane l handles rows 4l .. 4l + 3; the scales are loaded one K block ahead.
+template <int BN, bool kPair>
+__device__ void gemm_scales(const GemmSmem<BN, kPair>& sm, const GemmArgs& g, int tiles_m, int tiles_n,
+                            int num_tiles, int nkb, int t0, int dt) {
+  using Cfg = GemmCfg<BN, kPair>;
+  const int lane = threadIdx.x & 31;
+  const int nbw = (g.N + 127) >> 7;   // weight blocks along N
+  auto load = [&](int tl, int k, float (&a)[4], float (&w)[2]) {
+    int mt, nt;
+    tile_coords(tl, tiles_m, tiles_n, mt, nt);
+    const int r0 = mt * Cfg::TILE_M + 4 * lane;
+    const float* p = g.sA + (size_t)k * g.ldsA + r0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) a[i] = r0 + i < g.M ? __ldg(p + i) : 0.f;
+    const int nb = nt * (BN / 128);
+    w[0] = nb < nbw ? __ldg(g.sW + (size_t)nb * nkb + k) : 0.f;
+    w[1] = nb + 1 < nbw ? __ldg(g.sW + (size_t)(nb + 1) * nkb + k) : 0.f;
+  };
+  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sw[2] = {0.f, 0.f};
+  int tile = t0, kb = 0;
+  if (tile < num_tiles) load(tile, 0, sa, sw);
+  for (uint32_t cnt = 0; tile < num_tiles; ++cnt) {
+    int ntile = tile, nk = kb + 1;
+    if (nk == nkb) {
+      nk = 0;
+      ntile += dt;
+    }
+    float na[4] = {0.f, 0.f, 0.f, 0.f}, nw[2] = {0.f, 0.f};
+    if (ntile < num_tiles) load(ntile, nk, na, nw);
+    const uint32_t buf = cnt % Cfg::NBUF;
+    const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
+    if (!mbar_wait(sm.tempty(buf), aph ^ 1u, sm.abort_flag())) return;
+    st_shared_v4(sm.scale_slot(buf, 0) + lane * 16, sa[0] * sw[0], sa[1] * sw[0], sa[2] * sw[0], sa[3] * sw[0]);
+    st_shared_v4(sm.scale_slot(buf, 1) + lane * 16, sa[0] * sw[1], sa[1] * sw[1], sa[2] * sw[1], sa[3] * sw[1]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(sm.tfull(buf));   // release: the slot's stores come first
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sa[i] = na[i];
+    sw[0] = nw[0];
+    sw[1] = nw[1];
+    tile = ntile;
+    kb = nk;
+  }
+}
+
 template <int BN, bool kPair>
 __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base, const GemmArgs& g,
                               const CUtensorMap* tmC, const CUtensorMap* tmR, int tiles_m, int tiles_n,
@@ -248,8 +306,10 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
     cp_async_commit();
     ++pf_q;
   };
+  if constexpr (!Cfg::SCALE_WARP) {
 #pragma unroll 1
-  for (int i = 0; i < Cfg::SA_DEPTH - 1; ++i) prefetch_scale();
+    for (int i = 0; i < Cfg::SA_DEPTH - 1; ++i) prefetch_scale();
+  }
   uint32_t cnt = 0, it = 0;
   for (int tile = t0; tile < num_tiles; tile += dt, ++it) {
     int mt, nt;
@@ -280,18 +340,24 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
 #pragma unroll
     for (int j = 0; j < Cfg::NH * 32; ++j) acc[j] = 0ull;
     // the weight scale (the same for the whole warp, an L1 hit) is loaded one K block ahead
-    float sw_next = col_ok ? __ldg(sw_ptr) : 0.f;
+    float sw_next = 0.f;
+    if constexpr (!Cfg::SCALE_WARP) sw_next = col_ok ? __ldg(sw_ptr) : 0.f;
     for (int kb = 0; kb < nkb; ++kb, ++cnt) {
       const uint32_t buf = cnt % Cfg::NBUF;
       const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
-      cp_async_wait<Cfg::SA_DEPTH - 2>();
-      const float scale = ld_shared_f32(ring + (cnt & (Cfg::SA_DEPTH - 1)) * 128) * sw_next;
-      prefetch_scale();
-      if (kb + 1 < nkb) sw_next = col_ok ? __ldg(sw_ptr + kb + 1) : 0.f;
-      const uint64_t s2 = f2pack(scale, scale);
+      float scale;
+      if constexpr (!Cfg::SCALE_WARP) {
+        cp_async_wait<Cfg::SA_DEPTH - 2>();
+        scale = ld_shared_f32(ring + (cnt & (Cfg::SA_DEPTH - 1)) * 128) * sw_next;
+        prefetch_scale();
+        if (kb + 1 < nkb) sw_next = col_ok ? __ldg(sw_ptr + kb + 1) : 0.f;
+      }
       if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(4, cnt);  // epilogue: waiting for partial
       const bool ok = mbar_wait(sm.tfull(buf), aph, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
+      // (with the scale warp, tfull also covers the scale slot)
+      if constexpr (Cfg::SCALE_WARP) scale = ld_shared_f32(sm.scale_slot(buf, cg) + r_in * 4);
+      const uint64_t s2 = f2pack(scale, scale);
       if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(5, cnt);  // epilogue: partial ready
       tc_fence_after();
       const uint32_t taddr = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + cg * Cfg::COLS;
@@ -419,7 +485,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, kPair>::THREADS, 1)
       mbar_init(sm.empty(s), 1);
     }
     for (int b = 0; b < Cfg::NBUF; ++b) {
-      mbar_init(sm.tfull(b), 1);
+      mbar_init(sm.tfull(b), Cfg::SCALE_WARP ? 2 : 1);   // MMA commit (+ scale warp)
       mbar_init(sm.tempty(b), Cfg::TEMPTY_COUNT);
     }
     for (int w = 0; w < Cfg::EPI_WARPS; ++w) mbar_init(sm.res_full(w), 1);
@@ -450,6 +516,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, kPair>::THREADS, 1)
       gemm_producer<BN, kPair>(sm, &tmA, &tmB, tiles_m, tiles_n, num_tiles, nkb, t0, dt, rank);
     } else if (warp == 1 && lane == 0 && rank == 0) {
       gemm_mma<BN, kPair>(sm, tmem_base, num_tiles, nkb, t0, dt);
+    } else if (Cfg::SCALE_WARP && warp == 2) {
+      gemm_scales<BN, kPair>(sm, args, tiles_m, tiles_n, num_tiles, nkb, t0, dt);
     }
   } else {
     if (Cfg::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
