@@ -39,6 +39,10 @@ namespace {
 // BN = 256: 12 warps
 // (warpgroup 0 = TMA, MMA and two idle warps, which give registers away with
 // setmaxnreg; warpgroups 1-2 = 8 epilogue warps, one per 128 columns x 32 rows).
+#ifndef VITQ_SCALE_AHEAD
+#define VITQ_SCALE_AHEAD 2
+#endif
+
 template <int BN, bool kPair = false>
 struct GemmCfg {
   static constexpr int BM = 128, BK = 128;            // rows of A per CTA, K per stage
@@ -55,19 +59,21 @@ struct GemmCfg {
   static constexpr int NH = COLS / 64;                // 64-column halves per warp
   static constexpr int EPI_WARPS = (BN / COLS) * 4;
   static constexpr int TEMPTY_COUNT = EPI_WARPS * (kPair ? 2 : 1);   // both CTAs' epilogues free a buffer
+  // BN = 256 (single CTAs): warp 2 of warpgroup 0 (otherwise idle) stages each K
+  // block's combined scales sA * sW for the tile's 128 rows and its two weight blocks
+  // in a slot tied to the K block's TMEM buffer.  Otherwise each epilogue warp keeps
+  // its 32 rows' activation scales of the next SA_DEPTH K blocks in its own ring (at
+  // BN = 128 an extra scale warp measured slower: its K blocks are too short).
+  static constexpr bool SCALE_WARP = BN == 256 && !kPair;
+  static constexpr int SCALE_AHEAD = VITQ_SCALE_AHEAD;   // K blocks of scales in flight
   static constexpr int EPI_WARP0 = BN == 256 ? 4 : 2;
   static constexpr int THREADS = 32 * (EPI_WARP0 + EPI_WARPS);
   static constexpr bool SPLIT_REGS = BN == 256;
   static constexpr int MIN_LAUNCH_REGS = 168;   // 384 x 168 >= 128 x 56 + 256 x 224 (BN = 256)
   static constexpr int OUT_WARP_BYTES = NH * 4096;  // 64-column SW128 boxes of 32 rows
   static constexpr int OUT_BYTES = EPI_WARPS * (OUT_WARP_BYTES + COLS * 2);   // + the warp's bias values
-  // BN = 256 (single CTAs): warp 2, otherwise idle, stages each K block's combined
-  // scales sA * sW for the tile's 128 rows and two weight blocks in a slot tied to
-  // the K block's TMEM buffer.  Otherwise each epilogue warp keeps its 32 rows'
-  // activation scales of the next SA_DEPTH K blocks in its own ring.
-  static constexpr bool SCALE_WARP = BN == 256 && !kPair;
   static constexpr int SA_DEPTH = 8;
-  static constexpr int SA_BYTES = SCALE_WARP ? NBUF * 2 * 128 * 4 : EPI_WARPS * SA_DEPTH * 32 * 4;
+  static constexpr int SA_BYTES = SCALE_WARP ? NBUF * (BN / 128) * 128 * 4 : EPI_WARPS * SA_DEPTH * 32 * 4;
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * NBUF + EPI_WARPS) * 8 + 16;
   static constexpr size_t SMEM = (size_t)STAGES * STAGE_BYTES + OUT_BYTES + SA_BYTES + 1024 + BAR_BYTES;
 };
@@ -100,7 +106,7 @@ struct GemmSmem {
   }
   // combined scales of TMEM buffer b, weight block cb of the tile (128 rows, fp32)
   __device__ uint32_t scale_slot(int b, int cb) const {
-    return smem_u32(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES + (b * 2 + cb) * 512);
+    return smem_u32(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES + (b * (BN / 128) + cb) * 512);
   }
   __device__ uint32_t sa_ring(int w) const {
     return smem_u32(base + (size_t)Cfg::STAGES * Cfg::STAGE_BYTES + Cfg::OUT_BYTES + w * Cfg::SA_DEPTH * 128);
@@ -213,53 +219,62 @@ __device__ void gemm_mma(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base, int 
   }
 }
 
-// Scale producer (BN = 256): for each K block of this CTA's tiles, in the MMA's
-// order, sA[kb, m] * sW[n / 128, kb] for the tile's 128 rows and both weight blocks
-// into the slot of the K block's TMEM buffer, once the epilogue has released that
-// buffer (the tempty phase the MMA thread waits for); then one arrival on the
+// Scale producer (BN = 256): for each K block of this CTA's tiles, in the
+// MMA's order, sA[kb, m] * sW[n / 128, kb] for the tile's 128 rows and its weight
+// blocks into the slot of the K block's TMEM buffer, once the epilogue has released
+// that buffer (the tempty phase the MMA thread waits for); then one arrival on the
 // buffer's tfull barrier, which completes when this and the MMAs' commit have both
-// arrived.  Lane l handles rows 4l .. 4l + 3; the scales are loaded one K block ahead.
+// arrived.  Lane l handles rows 4l .. 4l + 3; the scales of the next SCALE_AHEAD
+// K blocks are in flight in registers (a ring indexed by the unrolled loop).
 template <int BN, bool kPair>
 __device__ void gemm_scales(const GemmSmem<BN, kPair>& sm, const GemmArgs& g, int tiles_m, int tiles_n,
                             int num_tiles, int nkb, int t0, int dt) {
   using Cfg = GemmCfg<BN, kPair>;
+  constexpr int WB = BN >= 128 ? BN / 128 : 1;   // weight blocks per tile
+  constexpr int L = Cfg::SCALE_AHEAD;
   const int lane = threadIdx.x & 31;
   const int nbw = (g.N + 127) >> 7;   // weight blocks along N
-  auto load = [&](int tl, int k, float (&a)[4], float (&w)[2]) {
+  if (t0 >= num_tiles) return;
+  const int total = ((num_tiles - t0 + dt - 1) / dt) * nkb;   // K blocks of this CTA
+  int ltile = t0, lkb = 0;                                     // next K block to load
+  auto load = [&](float (&a)[4], float (&w)[WB]) {
     int mt, nt;
-    tile_coords(tl, tiles_m, tiles_n, mt, nt);
+    tile_coords(ltile, tiles_m, tiles_n, mt, nt);
     const int r0 = mt * Cfg::TILE_M + 4 * lane;
-    const float* p = g.sA + (size_t)k * g.ldsA + r0;
+    const float* p = g.sA + (size_t)lkb * g.ldsA + r0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) a[i] = r0 + i < g.M ? __ldg(p + i) : 0.f;
-    const int nb = nt * (BN / 128);
-    w[0] = nb < nbw ? __ldg(g.sW + (size_t)nb * nkb + k) : 0.f;
-    w[1] = nb + 1 < nbw ? __ldg(g.sW + (size_t)(nb + 1) * nkb + k) : 0.f;
-  };
-  float sa[4] = {0.f, 0.f, 0.f, 0.f}, sw[2] = {0.f, 0.f};
-  int tile = t0, kb = 0;
-  if (tile < num_tiles) load(tile, 0, sa, sw);
-  for (uint32_t cnt = 0; tile < num_tiles; ++cnt) {
-    int ntile = tile, nk = kb + 1;
-    if (nk == nkb) {
-      nk = 0;
-      ntile += dt;
-    }
-    float na[4] = {0.f, 0.f, 0.f, 0.f}, nw[2] = {0.f, 0.f};
-    if (ntile < num_tiles) load(ntile, nk, na, nw);
-    const uint32_t buf = cnt % Cfg::NBUF;
-    const uint32_t aph = (cnt / Cfg::NBUF) & 1u;
-    if (!mbar_wait(sm.tempty(buf), aph ^ 1u, sm.abort_flag())) return;
-    st_shared_v4(sm.scale_slot(buf, 0) + lane * 16, sa[0] * sw[0], sa[1] * sw[0], sa[2] * sw[0], sa[3] * sw[0]);
-    st_shared_v4(sm.scale_slot(buf, 1) + lane * 16, sa[0] * sw[1], sa[1] * sw[1], sa[2] * sw[1], sa[3] * sw[1]);
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sm.tfull(buf));   // release: the slot's stores come first
 #pragma unroll
-    for (int i = 0; i < 4; ++i) sa[i] = na[i];
-    sw[0] = nw[0];
-    sw[1] = nw[1];
-    tile = ntile;
-    kb = nk;
+    for (int c = 0; c < WB; ++c) {
+      const int nb = nt * WB + c;
+      w[c] = nb < nbw ? __ldg(g.sW + (size_t)nb * nkb + lkb) : 0.f;
+    }
+    if (++lkb == nkb) {
+      lkb = 0;
+      ltile += dt;
+    }
+  };
+  float a[L][4], w[L][WB];
+#pragma unroll
+  for (int j = 0; j < L; ++j)
+    if (j < total) load(a[j], w[j]);
+  for (int cnt = 0; cnt < total;) {
+#pragma unroll
+    for (int j = 0; j < L; ++j) {
+      if (cnt < total) {
+        const uint32_t buf = (uint32_t)cnt % Cfg::NBUF;
+        const uint32_t aph = ((uint32_t)cnt / Cfg::NBUF) & 1u;
+        if (!mbar_wait(sm.tempty(buf), aph ^ 1u, sm.abort_flag())) return;
+#pragma unroll
+        for (int c = 0; c < WB; ++c)
+          st_shared_v4(sm.scale_slot(buf, c) + lane * 16, a[j][0] * w[j][c], a[j][1] * w[j][c], a[j][2] * w[j][c],
+                       a[j][3] * w[j][c]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sm.tfull(buf));   // release: the slot's stores come first
+        if (cnt + L < total) load(a[j], w[j]);
+        ++cnt;
+      }
+    }
   }
 }
 
@@ -356,7 +371,8 @@ __device__ void gemm_epilogue(const GemmSmem<BN, kPair>& sm, uint32_t tmem_base,
       const bool ok = mbar_wait(sm.tfull(buf), aph, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
       // (with the scale warp, tfull also covers the scale slot)
-      if constexpr (Cfg::SCALE_WARP) scale = ld_shared_f32(sm.scale_slot(buf, cg) + r_in * 4);
+      if constexpr (Cfg::SCALE_WARP)   // slot of this warp's weight block within the tile
+        scale = ld_shared_f32(sm.scale_slot(buf, (cg * Cfg::COLS) >> 7) + r_in * 4);
       const uint64_t s2 = f2pack(scale, scale);
       if (lane == 0 && warp == Cfg::EPI_WARP0) VITQ_TRACE_EV(5, cnt);  // epilogue: partial ready
       tc_fence_after();
@@ -516,8 +532,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, kPair>::THREADS, 1)
       gemm_producer<BN, kPair>(sm, &tmA, &tmB, tiles_m, tiles_n, num_tiles, nkb, t0, dt, rank);
     } else if (warp == 1 && lane == 0 && rank == 0) {
       gemm_mma<BN, kPair>(sm, tmem_base, num_tiles, nkb, t0, dt);
-    } else if (Cfg::SCALE_WARP && warp == 2) {
-      gemm_scales<BN, kPair>(sm, args, tiles_m, tiles_n, num_tiles, nkb, t0, dt);
+    } else if (warp == 2) {
+      if constexpr (Cfg::SCALE_WARP) gemm_scales<BN, kPair>(sm, args, tiles_m, tiles_n, num_tiles, nkb, t0, dt);
     }
   } else {
     if (Cfg::SPLIT_REGS) asm volatile("setmaxnreg.inc.sync.aligned.u32 224;" ::: "memory");
