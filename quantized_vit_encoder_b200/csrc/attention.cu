@@ -6,24 +6,30 @@
 // with cu_seqlens): O = softmax(Q K^T * scale) V per segment and head.
 //
 // Design (B200):
-//   * one CTA per (segment, head, 256 queries = two 128-row Q tiles); 20 warps:
-//     TMA producer, one MMA issuer per Q tile, and eight softmax warps per Q
-//     tile, two per TMEM lane quadrant (thread = query row = TMEM lane; each
-//     warp of a pair owns 64 of the tile's 128 score columns, and the pair
-//     combines its row maxima through shared memory).  S_x(j+1) is computed
-//     while the softmax of S_x(j) runs (the softmax frees S_x once it holds it
-//     in registers), and the two tiles interleave on the tensor core;
+//   * one CTA per (segment, head, 256 queries = two 128-row Q tiles); 12 warps:
+//     a TMA producer for K, one for V, one MMA issuer per Q tile, and four
+//     softmax warps per Q tile, one per TMEM lane quadrant (thread = query row =
+//     TMEM lane, owning all 128 score columns of its row, so the row max needs
+//     no exchange between warps).  S_x(j+1) is computed while the softmax of
+//     S_x(j) runs (the softmax frees S_x once it holds it in registers), and the
+//     two tiles interleave on the tensor core;
+//   * P is double-buffered per Q tile: the softmax writes P(j) into buffer j & 1
+//     while P(j-1).V may still be reading the other one, and waits only for
+//     P(j-2).V (per-buffer barriers, so no mbarrier phase can be confused with
+//     the next);
 //   * the softmax exponentials run on MUFU ex2; a share can move to a polynomial
 //     on the FMA pipe (kPolyEvery).  The softmax warps of tile A and tile B that
 //     share an SMSP take turns for their exponentials, so each turn has MUFU to
-//     itself while the other tile reads its next scores and waits for its P.V;
+//     itself while the other tile reads its next scores;
 //   * K and V are read straight from the packed qkv activation [n, 3, 16, 72]
 //     through 3D TMA maps (d, slot, token).  head_dim 72 is padded to 80 by
 //     the tensor map itself: d >= 72 lies outside the map so TMA fills zeros,
-//     and the padding never exists in HBM.  K: d 0..63 in a 128B-swizzled tile,
-//     d 64..79 in a 32B-swizzled tile.  V: d 0..63 and d 64..127 in two
-//     128B-swizzled tiles, so that P.V is one N = 80 MMA per 16 keys (two
-//     MMAs of N = 64 and 16 cost twice as much: each re-reads P);
+//     and the padding never exists in HBM.  K (a ring of two stages): d 0..63 in
+//     a 128B-swizzled tile, d 64..79 in a 32B-swizzled tile.  V (its own ring of
+//     two stages): five 32B-swizzled atoms of 16 dims, so that P.V is one N = 80
+//     MMA per 16 keys over 20 KB instead of two 64-wide 128B-swizzled atoms
+//     (32 KB), which is what leaves room for the second P buffers.  A K stage is
+//     freed by the S MMAs, a V stage by the P.V MMAs;
 //   * the softmax threads copy their Q rows into TMEM once (columns packed two
 //     bf16 per 32-bit column), and S = Q K^T runs as 5 tcgen05.mma with A in
 //     TMEM (K = 16 each) into the tile's TMEM S buffer;
@@ -40,21 +46,20 @@
 namespace vitq {
 namespace {
 
-constexpr int kBM = 128, kBN = 128, kStages = 3, kQTiles = 2;
-// Shared memory: a ring of K/V stages, the P tiles (A, B).
-constexpr int kKV0 = 0, kKVStride = 53248;
-constexpr int kKLo = 0, kKHi = 16384, kVLo = 20480, kVHi = 36864;   // V hi = V lo + 16384 (N-atom stride)
-constexpr int kP0 = kKV0 + kStages * kKVStride;         // P tile X: two 64-key atoms of 16 KB
+constexpr int kBM = 128, kBN = 128, kQTiles = 2, kKStages = 2, kVStages = 2;
+// Shared memory: a ring of K stages (d 0..63 in a 128B-swizzled tile, d 64..79 in a
+// 32B-swizzled tile), a ring of V stages (five 32B-swizzled atoms of 16 dims, so
+// that N = 80 spans them with one descriptor), and two P buffers per Q tile.
+constexpr int kKStride = 20480, kKHi = 16384;
+constexpr int kVStride = 20480, kVAtom = 4096;
+constexpr int kK0 = 0, kV0 = kK0 + kKStages * kKStride;
+constexpr int kP0 = kV0 + kVStages * kVStride;          // P buffer (x, b): two 64-key atoms of 16 KB
 constexpr int kPBytes = 32768;
-// Row-maximum exchange of the two softmax warps of a row quadrant:
-// [tile][step parity][half][128 rows] fp32 (the last exchange carries the row sums).
-constexpr int kRed = kP0 + kQTiles * kPBytes;
-constexpr int kBar = kRed + kQTiles * 2 * 2 * 128 * 4;
-// barriers: slot 0 (unused), kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2],
-// s_free[2], turn[2][4] (the softmax warps of tile x on SMSP q finished their
-// exponentials), q_ready[2] (Q tile x is in TMEM), pair[2][4] (both halves of
-// tile x, quadrant q, posted their partial row maxima)
-constexpr int kNumBars = 1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles + kQTiles * 4;
+constexpr int kBar = kP0 + kQTiles * 2 * kPBytes;
+// barriers: slot 0 (unused), k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2],
+// s_free[2], p_full[2][2], pv_done[2][2] (per Q tile and P buffer), turn[2][4] (the
+// softmax warp of tile x on SMSP q finished its exponentials), q_ready[2]
+constexpr int kNumBars = 1 + 2 * kKStages + 2 * kVStages + 2 * kQTiles + 4 * kQTiles + kQTiles * 4 + kQTiles;
 constexpr size_t kAttnSmem = 1024 + kBar + kNumBars * 8 + 16;
 static_assert(kAttnSmem <= 232448, "shared memory budget");
 // TMEM columns: S_A 0..127, S_B 128..255, O_A 256..335, Q_A 336..383, O_B 384..463,
@@ -62,10 +67,13 @@ static_assert(kAttnSmem <= 232448, "shared memory budget");
 __device__ __forceinline__ uint32_t tmem_s(int x) { return (uint32_t)x * 128u; }
 __device__ __forceinline__ uint32_t tmem_o(int x) { return 256u + (uint32_t)x * 128u; }
 __device__ __forceinline__ uint32_t tmem_q(int x) { return 336u + (uint32_t)x * 128u; }
-// Warpgroup 0: warp 0 TMA producer, warps 1 and 2 MMA issuers for Q tiles A
-// and B (warp 3 idle); warps 4-11 softmax of Q tile A, 12-19 of Q tile B (two
-// warps per TMEM lane quadrant, each owning 64 of the 128 score columns).
-constexpr int kThreads = 128 + 256 * kQTiles;
+// Warpgroup 0: warp 0 the K producer, warps 1 and 2 the MMA issuers for Q tiles A
+// and B, warp 3 the V producer; warps 4-7 the softmax of Q tile A, 8-11 of Q tile B
+// (one per TMEM lane quadrant).
+constexpr int kThreads = 128 + 128 * kQTiles;
+// register split: warpgroup 0 (TMA, MMA) 56 per thread, the softmax warpgroups 208
+constexpr int kAttnMinLaunchRegs = 158;
+static_assert(kThreads * kAttnMinLaunchRegs >= 128 * 56 + 256 * 208, "register split");
 // Share of the softmax exponentials moved from MUFU to the FMA-pipe polynomial:
 // one pair in kPolyEvery (0 = none).  MUFU ex2 runs at 16 per clock per SM.
 #ifndef VITQ_ATTN_POLY_EVERY
@@ -73,9 +81,9 @@ constexpr int kThreads = 128 + 256 * kQTiles;
 #endif
 constexpr int kPolyEvery = VITQ_ATTN_POLY_EVERY;
 constexpr int kPolyMod = kPolyEvery > 0 ? kPolyEvery : 1;
-// 8-key group of the exponential loop after which the turn passes to the other tile (7 = at the end).
+// 8-key group of the exponential loop (16 per step) after which the turn passes to the other tile (15 = at the end).
 #ifndef VITQ_ATTN_TURN_AT
-#define VITQ_ATTN_TURN_AT 5
+#define VITQ_ATTN_TURN_AT 11
 #endif
 constexpr int kTurnAt = VITQ_ATTN_TURN_AT;
 // Whether the two tiles' softmax warps of one SMSP take turns for the exponentials.
@@ -108,26 +116,24 @@ struct AttnSmem {
   uint8_t* base;
   __device__ uint32_t at(int off) const { return smem_u32(base + off); }
   __device__ uint64_t* bar(int i) const { return reinterpret_cast<uint64_t*>(base + kBar) + i; }
-  __device__ uint32_t q_ready(int x) const { return smem_u32(bar(1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + x)); }
-  __device__ uint32_t kv_full(int s) const { return smem_u32(bar(1 + s)); }
-  __device__ uint32_t kv_empty(int s) const { return smem_u32(bar(1 + kStages + s)); }
-  __device__ uint32_t s_full(int x) const { return smem_u32(bar(1 + 2 * kStages + x)); }
-  __device__ uint32_t p_full(int x) const { return smem_u32(bar(1 + 2 * kStages + kQTiles + x)); }
-  __device__ uint32_t pv_done(int x) const { return smem_u32(bar(1 + 2 * kStages + 2 * kQTiles + x)); }
-  __device__ uint32_t s_free(int x) const { return smem_u32(bar(1 + 2 * kStages + 3 * kQTiles + x)); }
-  __device__ uint32_t turn(int x, int q) const { return smem_u32(bar(1 + 2 * kStages + 4 * kQTiles + x * 4 + q)); }
-  __device__ uint32_t pair(int x, int q) const {
-    return smem_u32(bar(1 + 2 * kStages + 4 * kQTiles + kQTiles * 4 + kQTiles + x * 4 + q));
-  }
-  __device__ float* red(int x, int par, int h) const {
-    return reinterpret_cast<float*>(base + kRed) + ((x * 2 + par) * 2 + h) * 128;
-  }
+  __device__ uint32_t k_full(int s) const { return smem_u32(bar(1 + s)); }
+  __device__ uint32_t k_empty(int s) const { return smem_u32(bar(1 + kKStages + s)); }
+  __device__ uint32_t v_full(int s) const { return smem_u32(bar(1 + 2 * kKStages + s)); }
+  __device__ uint32_t v_empty(int s) const { return smem_u32(bar(1 + 2 * kKStages + kVStages + s)); }
+  static constexpr int kB0 = 1 + 2 * kKStages + 2 * kVStages;
+  __device__ uint32_t s_full(int x) const { return smem_u32(bar(kB0 + x)); }
+  __device__ uint32_t s_free(int x) const { return smem_u32(bar(kB0 + kQTiles + x)); }
+  __device__ uint32_t p_full(int x, int b) const { return smem_u32(bar(kB0 + 2 * kQTiles + x * 2 + b)); }
+  __device__ uint32_t pv_done(int x, int b) const { return smem_u32(bar(kB0 + 4 * kQTiles + x * 2 + b)); }
+  __device__ uint32_t turn(int x, int q) const { return smem_u32(bar(kB0 + 6 * kQTiles + x * 4 + q)); }
+  __device__ uint32_t q_ready(int x) const { return smem_u32(bar(kB0 + 10 * kQTiles + x)); }
   __device__ uint32_t* tmem_holder() const { return reinterpret_cast<uint32_t*>(bar(kNumBars)); }
   __device__ volatile int* abort_flag() const {
     return reinterpret_cast<volatile int*>(tmem_holder() + 1);
   }
-  __device__ uint32_t kv(int s, int part) const { return at(kKV0 + s * kKVStride + part); }
-  __device__ uint32_t p(int x) const { return at(kP0 + x * kPBytes); }
+  __device__ uint32_t k(int s) const { return at(kK0 + s * kKStride); }
+  __device__ uint32_t v(int s) const { return at(kV0 + s * kVStride); }
+  __device__ uint32_t p(int x, int b) const { return at(kP0 + (x * 2 + b) * kPBytes); }
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -157,63 +163,79 @@ __device__ __forceinline__ float2 ex2_poly2(float x0, float x1) {
 
 
 
-__device__ void attn_producer(const AttnSmem& sm, const CUtensorMap* tlo, const CUtensorMap* thi,
-                              int head, int kv_row0, int n_kv, int off) {
+// K tiles (warp 0) and V tiles (warp 3) come from the packed qkv activation
+// through 3D maps (d, slot, token); d >= 72 lies outside the map and reads zero.
+// A K stage is free once both tiles' S MMAs of it have completed, a V stage once
+// both tiles' P.V MMAs have.
+__device__ void attn_load_k(const AttnSmem& sm, const CUtensorMap* tlo, const CUtensorMap* thi, int head,
+                            int kv_row0, int n_kv, int off) {
   for (int j = 0; j < n_kv; ++j) {
-    const int s = j % kStages;
-    const uint32_t ph = (uint32_t)(j / kStages) & 1u;
-    if (!mbar_wait(sm.kv_empty(s), ph ^ 1u, sm.abort_flag())) return;
-    mbar_arrive_expect_tx(sm.kv_full(s), kKVStride);
+    const int s = j % kKStages;
+    const uint32_t ph = (uint32_t)(j / kKStages) & 1u;
+    if (!mbar_wait(sm.k_empty(s), ph ^ 1u, sm.abort_flag())) return;
+    mbar_arrive_expect_tx(sm.k_full(s), kKStride);
     const int row = kv_row0 + kv_tile(j, off, n_kv) * kBN;
-    tma_load_3d(sm.kv(s, kKLo), tlo, 0, 16 + head, row, sm.kv_full(s));
-    tma_load_3d(sm.kv(s, kKHi), thi, 64, 16 + head, row, sm.kv_full(s));
-    tma_load_3d(sm.kv(s, kVLo), tlo, 0, 32 + head, row, sm.kv_full(s));
-    tma_load_3d(sm.kv(s, kVHi), tlo, 64, 32 + head, row, sm.kv_full(s));   // d 64..127, >= 72 zero
+    tma_load_3d(sm.k(s), tlo, 0, 16 + head, row, sm.k_full(s));
+    tma_load_3d(sm.k(s) + kKHi, thi, 64, 16 + head, row, sm.k_full(s));
+  }
+}
+__device__ void attn_load_v(const AttnSmem& sm, const CUtensorMap* thi, int head, int kv_row0, int n_kv,
+                            int off) {
+  for (int j = 0; j < n_kv; ++j) {
+    const int s = j % kVStages;
+    const uint32_t ph = (uint32_t)(j / kVStages) & 1u;
+    if (!mbar_wait(sm.v_empty(s), ph ^ 1u, sm.abort_flag())) return;
+    mbar_arrive_expect_tx(sm.v_full(s), kVStride);
+    const int row = kv_row0 + kv_tile(j, off, n_kv) * kBN;
+#pragma unroll
+    for (int a = 0; a < 5; ++a) tma_load_3d(sm.v(s) + a * kVAtom, thi, 16 * a, 32 + head, row, sm.v_full(s));
   }
 }
 
 // S_x = Q_x K_j^T (5 MMAs of K = 16 over the padded head_dim 80, Q from TMEM) into S buffer x.
 __device__ bool attn_issue_s(const AttnSmem& sm, uint32_t tmem, int x, int j) {
   constexpr uint32_t idesc = make_idesc(1, 1, 0, 0, 128, 128);
-  const int s = j % kStages;
-  if (!mbar_wait(sm.kv_full(s), (uint32_t)(j / kStages) & 1u, sm.abort_flag())) return false;
+  const int s = j % kKStages;
+  if (!mbar_wait(sm.k_full(s), (uint32_t)(j / kKStages) & 1u, sm.abort_flag())) return false;
   tc_fence_after();
   const uint32_t d = tmem + tmem_s(x), q = tmem + tmem_q(x);
-  const uint32_t klo = sm.kv(s, kKLo);
+  const uint32_t klo = sm.k(s);
 #pragma unroll
   for (int k = 0; k < 4; ++k)
     mma_bf16_ts(d, q + 8 * k, make_smem_desc(klo + 32 * k, 16, 1024, kSwizzle128B), idesc, k > 0 ? 1u : 0u);
-  mma_bf16_ts(d, q + 32, make_smem_desc(sm.kv(s, kKHi), 16, 256, kSwizzle32B), idesc, 1u);
+  mma_bf16_ts(d, q + 32, make_smem_desc(klo + kKHi, 16, 256, kSwizzle32B), idesc, 1u);
   tc_commit(sm.s_full(x));
+  tc_commit(sm.k_empty(s));
   return true;
 }
 
-// O_x += P_x V_j: P from shared memory (K-major), V MN-major in two 64-wide
-// atoms (LBO 16384 bytes apart); one N = 80 MMA per 16 keys.
+// O_x += P_x(j) V_j: P from shared memory (K-major, buffer j & 1), V MN-major in
+// five 16-wide 32B-swizzled atoms (LBO 4096 bytes apart); one N = 80 MMA per 16 keys.
 template <bool kVF16>
 __device__ bool attn_issue_pv(const AttnSmem& sm, uint32_t tmem, int x, int j) {
   constexpr uint32_t fmt = kVF16 ? 0u : 1u;
   constexpr uint32_t idesc = make_idesc(fmt, fmt, 0, 1, 128, 80);
-  if (!mbar_wait(sm.p_full(x), (uint32_t)j & 1u, sm.abort_flag())) return false;
+  const int b = j & 1;
+  if (!mbar_wait(sm.p_full(x, b), (uint32_t)(j >> 1) & 1u, sm.abort_flag())) return false;
+  const int s = j % kVStages;
+  if (!mbar_wait(sm.v_full(s), (uint32_t)(j / kVStages) & 1u, sm.abort_flag())) return false;
   VITQ_TRACE_EV(14 + x, j);   // mma: P complete
   tc_fence_after();
-  const int s = j % kStages;
-  const uint32_t vlo = sm.kv(s, kVLo), p0 = sm.p(x);
+  const uint32_t vb = sm.v(s), p0 = sm.p(x, b);
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const uint64_t ad = make_smem_desc(p0 + (k >> 2) * 16384 + (k & 3) * 32, 16, 1024, kSwizzle128B);
     const uint32_t acc = (j > 0 || k > 0) ? 1u : 0u;
-    mma_bf16_ss(tmem + tmem_o(x), ad, make_smem_desc(vlo + k * 2048, kVHi - kVLo, 1024, kSwizzle128B), idesc, acc);
+    mma_bf16_ss(tmem + tmem_o(x), ad, make_smem_desc(vb + k * 512, kVAtom, 256, kSwizzle32B), idesc, acc);
   }
-  tc_commit(sm.pv_done(x));
+  tc_commit(sm.pv_done(x, b));
+  tc_commit(sm.v_empty(s));
   return true;
 }
 
 // Tensor-core work of Q tile x, issued by its own thread.  S_x(j+1) is issued as
 // soon as the softmax has moved S_x(j) into registers (s_free), so it overlaps
-// that softmax; P_x(j).V_j follows when P_x(j) is in shared memory.  The two
-// tiles' threads interleave on the tensor core; a K/V stage is released when
-// both tiles' P.V of that stage have completed (kv_empty counts one commit per tile).
+// that softmax; P_x(j).V_j follows when P_x(j) is in shared memory.
 template <bool kVF16>
 __device__ void attn_mma(const AttnSmem& sm, uint32_t tmem, int x, int n_kv) {
   if (!mbar_wait(sm.q_ready(x), 0, sm.abort_flag())) return;
@@ -229,7 +251,6 @@ __device__ void attn_mma(const AttnSmem& sm, uint32_t tmem, int x, int n_kv) {
     }
     if (!attn_issue_pv<kVF16>(sm, tmem, x, j)) return;
     VITQ_TRACE_EV(12 + x, j);     // mma: P.V issued
-    tc_commit(sm.kv_empty(j % kStages));
   }
 }
 
@@ -241,23 +262,22 @@ __device__ __forceinline__ uint32_t pack_p(float lo, float hi, bool f16) {
   return pack_bf16x2(lo, hi);
 }
 
-// Two warps per (Q tile, TMEM lane quadrant); thread = query row = TMEM lane.
-// Half h of the pair owns score columns 64h..64h+63 of its rows and P atom h.
-// The halves combine their row maxima through shared memory every step (so
-// both follow the same running max); the row sums stay partial until the end.
-// Half 0 also copies the Q rows into TMEM, rescales O and writes the output.
+// One warp per (Q tile, TMEM lane quadrant); thread = query row = TMEM lane,
+// owning all 128 score columns of its row, so the row max needs no exchange
+// between warps.  The warp copies its Q rows into TMEM, rescales its O rows and
+// writes their output.
 template <bool kVF16>
-__device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& g, int x, int h, int n_q,
+__device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& g, int x, int n_q,
                              int head, int seq_start, int seq_len, int q0, int n_kv, int off) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quad = warp & 3;
   const int r = quad * 32 + lane;
   const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-  const uint32_t s_addr = tmem + lane_addr + tmem_s(x) + 64 * h, o_addr = tmem + lane_addr + tmem_o(x);
-  uint8_t* pbase = sm.base + kP0 + x * kPBytes + h * 16384;
-  const bool tr = h == 0 && quad == 0 && lane == 0;
+  const uint32_t s_addr = tmem + lane_addr + tmem_s(x), o_addr = tmem + lane_addr + tmem_o(x);
+  uint8_t* pbase0 = sm.base + kP0 + x * 2 * kPBytes;
+  const bool tr = quad == 0 && lane == 0;
   (void)tr;
-  if (h == 0) {
+  {
     // this thread's Q row -> TMEM (bf16 pairs in columns 0..35, zeros up to 47)
     const bool q_ok = q0 + r < seq_len && seq_start + q0 + r < g.n_tokens;
     const uint4* src = reinterpret_cast<const uint4*>(g.qkv + (size_t)(seq_start + q0 + r) * 3456 + head * 72);
@@ -286,41 +306,40 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
     if (!__all_sync(0xffffffffu, ok)) return;
     if (tr) VITQ_TRACE_EV(20 + x, j);   // softmax: S ready
     tc_fence_after();
-    // keys of this tile inside the segment, counted from this half's first column
-    const int valid = seq_len - kv_tile(j, off, n_kv) * kBN - 64 * h;
-    uint32_t su[2][32];
+    // keys of this tile inside the segment
+    const int valid = seq_len - kv_tile(j, off, n_kv) * kBN;
+    uint32_t su[4][32];
     tmem_ld32(s_addr, su[0]);
     tmem_ld32(s_addr + 32, su[1]);
+    tmem_ld32(s_addr + 64, su[2]);
+    tmem_ld32(s_addr + 96, su[3]);
     tmem_wait_ld();
     if (tr) VITQ_TRACE_EV(26 + x, j);   // softmax: S in registers
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(sm.s_free(x));
-    if (valid < 64) {
+    if (valid < kBN) {
 #pragma unroll
-      for (int i = 0; i < 64; ++i)
+      for (int i = 0; i < kBN; ++i)
         if (i >= valid) su[i >> 5][i & 31] = 0xFF800000u;   // -inf
     }
-    // partial row max: 8 independent chains of 3-input max, then a tree
+    // row max: 8 independent chains of 3-input max, then a tree
     float mp[8];
 #pragma unroll
     for (int k = 0; k < 8; ++k) mp[k] = __uint_as_float(su[0][k]);
 #pragma unroll
-    for (int i = 8; i < 64; i += 16)
+    for (int i = 8; i < kBN; i += 16)
 #pragma unroll
       for (int k = 0; k < 8; ++k)
         mp[k] = fmax3(mp[k], __uint_as_float(su[(i + k) >> 5][(i + k) & 31]),
                       __uint_as_float(su[(i + 8 + k) >> 5][(i + 8 + k) & 31]));
-    const float pm = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7]));
-    sm.red(x, j & 1, h)[r] = pm;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(sm.pair(x, quad));
-    ok = mbar_wait(sm.pair(x, quad), (uint32_t)j & 1u, sm.abort_flag());
-    if (!__all_sync(0xffffffffu, ok)) return;
-    const float mx = fmaxf(pm, sm.red(x, j & 1, 1 - h)[r]) * g.scale_log2;
-    if (j > 0) {
-      // P(j) overwrites P(j-1), and half 0 may rescale O: P(j-1).V must be done
-      ok = mbar_wait(sm.pv_done(x), (uint32_t)(j - 1) & 1u, sm.abort_flag());
+    const float mx = fmax3(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], mp[5]), fmaxf(mp[6], mp[7])) *
+                     g.scale_log2;
+    // P(j) goes to buffer j & 1, which P(j-2).V must have finished reading
+    const int pb = j & 1;
+    uint8_t* pbase = pbase0 + pb * kPBytes;
+    if (j >= 2) {
+      ok = mbar_wait(sm.pv_done(x, pb), (uint32_t)((j - 2) >> 1) & 1u, sm.abort_flag());
       if (!__all_sync(0xffffffffu, ok)) return;
       tc_fence_after();
     }
@@ -328,7 +347,6 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
     // new running max: it changes only when the tile max exceeds it by more than 8
     // (so P <= 2^8), and the decision is warp-uniform because the O rescale uses
     // warp-collective tcgen05.ld/st (rows that keep their max get alpha = 1).
-    // Both halves see the same maxima, so they take the same decisions.
     float alpha = 1.f;
     bool rescale = false;
     if (j == 0) {
@@ -349,12 +367,12 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
       if (!__all_sync(0xffffffffu, ok)) return;
     }
     if (tr) VITQ_TRACE_EV(28 + x, j);   // softmax: turn for the exponentials
-    // P = 2^(s * scale_log2 - m_run), rounded to the P.V operand type, into this
-    // half's 64-key atom of the swizzled P tile; 8 fp32 partial row sums.
+    // P = 2^(s * scale_log2 - m_run), rounded to the P.V operand type, into the
+    // two 64-key atoms of the swizzled P tile; 8 fp32 partial row sums.
     const uint64_t sc2 = f2pack(g.scale_log2, g.scale_log2), nm2 = f2pack(-m_run, -m_run);
     uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < kBN / 8; ++c) {
       uint32_t w[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -362,7 +380,6 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
         const float2 t = f2unpack(ffma2(f2pack(__uint_as_float(su[k0 >> 5][k0 & 31]),
                                                __uint_as_float(su[(k0 + 1) >> 5][(k0 + 1) & 31])),
                                         sc2, nm2));
-        // every kPolyEvery-th pair runs the FMA-pipe polynomial, the rest MUFU ex2
         float2 p;
         if (kPolyEvery > 0 && (i % kPolyMod) == kPolyMod - 1) {
           p = ex2_poly2(t.x, t.y);
@@ -373,7 +390,7 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
         w[i] = pack_p(p.x, p.y, kVF16);
         ls[i] = fadd2(ls[i], f2pack(p.x, p.y));
       }
-      uint8_t* dst = pbase + r * 128 + ((c ^ (r & 7)) << 4);
+      uint8_t* dst = pbase + (c >> 3) * 16384 + r * 128 + (((c & 7) ^ (r & 7)) << 4);
       *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
       // hand the turn to the other tile a little before the end, so that its
       // exponentials start while these finish (hides the hand-over latency)
@@ -382,8 +399,12 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
         if (lane == 0) mbar_arrive(sm.turn(x, quad));
       }
     }
-    if (rescale && h == 0) {
-      // O (complete up to P.V(j-1)) to the new max; done after P so the scores are dead
+    if (rescale) {
+      // O to the new max once P.V(j-1) has completed (it is read and written here);
+      // done after P so the scores are dead
+      ok = mbar_wait(sm.pv_done(x, (j - 1) & 1), (uint32_t)((j - 1) >> 1) & 1u, sm.abort_flag());
+      if (!__all_sync(0xffffffffu, ok)) return;
+      tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < 5; ++c) {
         uint32_t u[16];
@@ -403,19 +424,13 @@ __device__ void attn_softmax(const AttnSmem& sm, uint32_t tmem, const AttnArgs& 
     tc_fence_before();
     __syncwarp();
     if (tr) VITQ_TRACE_EV(24 + x, j);   // softmax: P written
-    if (lane == 0) mbar_arrive(sm.p_full(x));
+    if (lane == 0) mbar_arrive(sm.p_full(x, pb));
   }
-  bool ok = mbar_wait(sm.pv_done(x), (uint32_t)(n_kv - 1) & 1u, sm.abort_flag());
+  // the last P.V's commit tracks every earlier MMA of the tile
+  bool ok = mbar_wait(sm.pv_done(x, (n_kv - 1) & 1), (uint32_t)((n_kv - 1) >> 1) & 1u, sm.abort_flag());
   if (!__all_sync(0xffffffffu, ok)) return;
   tc_fence_after();
-  // row sum = the two halves' partial sums (one more exchange, slot parity n_kv)
-  sm.red(x, n_kv & 1, h)[r] = l_run;
-  __syncwarp();
-  if (lane == 0) mbar_arrive(sm.pair(x, quad));
-  ok = mbar_wait(sm.pair(x, quad), (uint32_t)n_kv & 1u, sm.abort_flag());
-  if (!__all_sync(0xffffffffu, ok)) return;
-  if (h != 0) return;
-  const float l_sum = l_run + sm.red(x, n_kv & 1, 1)[r];
+  const float l_sum = l_run;
   // O / l in 16-column chunks (columns 72..79 are the zero padding and are not stored)
   const bool row_ok = q0 + r < seq_len && seq_start + q0 + r < g.n_tokens;
   const float inv = 1.0f / l_sum;
@@ -457,18 +472,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   sm.base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(sm.kv_full(s), 1);
-      mbar_init(sm.kv_empty(s), (uint32_t)n_q);       // one commit per active Q tile
+    for (int s = 0; s < kKStages; ++s) {
+      mbar_init(sm.k_full(s), 1);
+      mbar_init(sm.k_empty(s), (uint32_t)n_q);       // one commit per active Q tile
+    }
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(sm.v_full(s), 1);
+      mbar_init(sm.v_empty(s), (uint32_t)n_q);
     }
     for (int x = 0; x < kQTiles; ++x) {
-      for (int q = 0; q < 4; ++q) mbar_init(sm.turn(x, q), 2);
-      for (int q = 0; q < 4; ++q) mbar_init(sm.pair(x, q), 2);
+      for (int q = 0; q < 4; ++q) mbar_init(sm.turn(x, q), 1);
       mbar_init(sm.q_ready(x), 4);
       mbar_init(sm.s_full(x), 1);
-      mbar_init(sm.p_full(x), 8);
-      mbar_init(sm.pv_done(x), 1);
-      mbar_init(sm.s_free(x), 8);
+      mbar_init(sm.s_free(x), 4);
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(sm.p_full(x, b), 4);
+        mbar_init(sm.pv_done(x, b), 1);
+      }
     }
     *sm.abort_flag() = 0;
     fence_barrier_init();
@@ -483,17 +503,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();   // inputs may be the previous kernel's outputs
   const uint32_t tmem = *sm.tmem_holder();
   if (warp < 4) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
     if (warp == 0 && lane == 0) {
       prefetch_tensormap(&tlo);
       prefetch_tensormap(&thi);
-      attn_producer(sm, &tlo, &thi, head, seq_start, n_kv, off);
+      attn_load_k(sm, &tlo, &thi, head, seq_start, n_kv, off);
+    } else if (warp == 3 && lane == 0) {
+      prefetch_tensormap(&thi);
+      attn_load_v(sm, &thi, head, seq_start, n_kv, off);
     } else if ((warp == 1 || warp == 2) && lane == 0 && warp - 1 < n_q) {
       attn_mma<kVF16>(sm, tmem, warp - 1, n_kv);
     }
   } else {
-    const int x = (warp - 4) >> 3, h = ((warp - 4) >> 2) & 1;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 208;" ::: "memory");
+    const int x = (warp - 4) >> 2;
     if (x < n_q)
-      attn_softmax<kVF16>(sm, tmem, args, x, h, n_q, head, seq_start, seq_len, q0 + x * kBM, n_kv, off);
+      attn_softmax<kVF16>(sm, tmem, args, x, n_q, head, seq_start, seq_len, q0 + x * kBM, n_kv, off);
   }
   tc_fence_before();
   __syncthreads();
@@ -518,6 +543,14 @@ cudaError_t launch_attention(const __nv_bfloat16* qkv, int n_tokens, const int32
   auto kern = v_f16 ? attn_kernel<true> : attn_kernel<false>;
   e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kAttnSmem);
   if (e != cudaSuccess) return e;
+  {
+    // setmaxnreg.inc only draws on the registers the CTA was launched with:
+    // 384 x launch >= 128 x 56 + 256 x 208 needs launch >= 158
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs < kAttnMinLaunchRegs) return cudaErrorInvalidConfiguration;
+  }
   AttnArgs a{qkv, cu, out, n_tokens, scale * 1.4426950408889634f};
   dim3 grid((max_seqlen + kBM * kQTiles - 1) / (kBM * kQTiles), 16, n_seqs);
   return launch_pdl(kern, grid, dim3(kThreads), kAttnSmem, st, tlo, thi, a);
