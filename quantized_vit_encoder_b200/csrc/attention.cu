@@ -19,8 +19,8 @@
 //     the next);
 //   * the softmax exponentials run on MUFU ex2; a share can move to a polynomial
 //     on the FMA pipe (kPolyEvery).  The softmax warps of tile A and tile B that
-//     share an SMSP take turns for their exponentials, so each turn has MUFU to
-//     itself while the other tile reads its next scores;
+//     share an SMSP may take turns for their exponentials (VITQ_ATTN_TURNS=1, off:
+//     with two P buffers per tile both tiles' warps running at once is faster);
 //   * K and V are read straight from the packed qkv activation [n, 3, 16, 72]
 //     through 3D TMA maps (d, slot, token).  head_dim 72 is padded to 80 by
 //     the tensor map itself: d >= 72 lies outside the map so TMA fills zeros,
@@ -86,9 +86,10 @@ constexpr int kPolyMod = kPolyEvery > 0 ? kPolyEvery : 1;
 #define VITQ_ATTN_TURN_AT 11
 #endif
 constexpr int kTurnAt = VITQ_ATTN_TURN_AT;
-// Whether the two tiles' softmax warps of one SMSP take turns for the exponentials.
+// Whether the two tiles' softmax warps of one SMSP take turns for the exponentials
+// (with two P buffers per tile the turns measured slower: 278 vs 271 us at 6256 tokens).
 #ifndef VITQ_ATTN_TURNS
-#define VITQ_ATTN_TURNS 1
+#define VITQ_ATTN_TURNS 0
 #endif
 constexpr bool kTakeTurns = VITQ_ATTN_TURNS != 0;
 
