@@ -104,8 +104,10 @@ def attention(lib):
     vitq.attention_varlen(qkv, cu, n, out=out, flags=vitq.V_FP16)
     torch.cuda.synchronize()
     t = read_table(lib)
-    R = range(10, 90)
-    print("tile A step period (S ready to S ready, 64 keys):", _med([t[20, j + 1] - t[20, j] for j in R]))
+    steps = int((t[20] > 0).sum())            # 128-key steps recorded for tile A
+    R = range(2, max(3, steps - 2))
+    print(f"{steps} steps; tile A step period (S ready to S ready, 128 keys):",
+          _med([t[20, j + 1] - t[20, j] for j in R]))
     print("exponential phase (turn -> P written): A", _med([t[24, j] - t[28, j] for j in R]),
           "B", _med([t[25, j] - t[29, j] for j in R]))
     print("S ready -> S in registers", _med([t[26, j] - t[20, j] for j in R]),
